@@ -1,0 +1,80 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module draws random numbers and nothing else: it holds none of the
+attention arithmetic, so the GPU library and the oracle can both be fed from it
+without sharing any computation.
+
+Recipe (one ``torch.Generator('cpu')`` per workload, seeded with the workload's
+seed): draw, in this order, the per-sequence cache lengths (decode only), then
+Q, K, V and, for the backward, dO, each as float32 N(0, 1) of the full tensor
+shape; multiply Q by ``q_scale`` (4 for the peaky-row workload); round every
+tensor to bfloat16 with round-to-nearest-even (``Tensor.to``).  Layout is
+contiguous [B, H, L, d]; caches are [B, H, cap, d].
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass
+class AttentionInputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    dO: torch.Tensor | None = None
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor
+    kcache: torch.Tensor
+    vcache: torch.Tensor
+    kv_lens: torch.Tensor
+
+
+def _normal(gen: torch.Generator, shape) -> torch.Tensor:
+    return torch.randn(*shape, generator=gen, dtype=torch.float32)
+
+
+def attention_inputs(B: int, H: int, Lq: int, Lk: int, d: int, seed: int, q_scale: float = 1.0,
+                     with_dO: bool = False) -> AttentionInputs:
+    """bf16 CPU tensors Q [B,H,Lq,d], K/V [B,H,Lk,d] (and dO [B,H,Lq,d])."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    q = (_normal(gen, (B, H, Lq, d)) * q_scale).to(torch.bfloat16)
+    k = _normal(gen, (B, H, Lk, d)).to(torch.bfloat16)
+    v = _normal(gen, (B, H, Lk, d)).to(torch.bfloat16)
+    dO = _normal(gen, (B, H, Lq, d)).to(torch.bfloat16) if with_dO else None
+    return AttentionInputs(q, k, v, dO)
+
+
+def decode_inputs(B: int, H: int, cap: int, d: int, seed: int, len_lo: int, len_hi: int) -> DecodeInputs:
+    """Decode workload: kv_lens ~ U{len_lo..len_hi} (int32 [B]), q [B,H,d], caches [B,H,cap,d].
+
+    Every cache slot holds N(0,1) data, including slots past a sequence's
+    length (a poison test overwrites those separately).
+    """
+    gen = torch.Generator("cpu").manual_seed(seed)
+    kv_lens = torch.randint(len_lo, len_hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    q = _normal(gen, (B, H, d)).to(torch.bfloat16)
+    kc = torch.empty((B, H, cap, d), dtype=torch.bfloat16)
+    vc = torch.empty((B, H, cap, d), dtype=torch.bfloat16)
+    # Drawn one sequence at a time to bound the float32 temporaries.
+    for b in range(B):
+        kc[b] = _normal(gen, (H, cap, d)).to(torch.bfloat16)
+    for b in range(B):
+        vc[b] = _normal(gen, (H, cap, d)).to(torch.bfloat16)
+    return DecodeInputs(q, kc, vc, kv_lens)
+
+
+# The workloads the library is measured and checked on.  Shapes and value
+# distributions follow the pages' sizes: the 4,096-token example, a training
+# shape at 8,192, a 65,536-token context and a decode batch over a long cache.
+WORKLOADS = {
+    "tiny_fwd": dict(kind="fwd", B=1, H=2, L=256, d=64, causal=False, q_scale=1.0, seed=1),
+    "fwd_L4096_peaky": dict(kind="fwd", B=4, H=16, L=4096, d=128, causal=True, q_scale=4.0, seed=2),
+    "train_L8192": dict(kind="fwdbwd", B=2, H=16, L=8192, d=128, causal=True, q_scale=1.0, seed=3),
+    "long_L65536": dict(kind="fwd", B=1, H=8, L=65536, d=128, causal=True, q_scale=1.0, seed=4),
+    "decode_cap32768": dict(kind="decode", B=64, H=32, cap=32768, d=128, len_lo=1024, len_hi=32768, seed=5),
+}

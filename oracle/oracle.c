@@ -1,0 +1,361 @@
+/*
+ * Reference ("oracle") implementation of exact scaled-dot-product attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow definition of what the
+ * GPU library computes, in double precision, so that the GPU results can be
+ * checked against it.  Only the test suite, the smoke check and the CPU-baseline
+ * leg of the benchmark may load it.  The product path never calls it and has no
+ * CPU fallback.  It shares no code, header or constant with the CUDA sources.
+ *
+ * Sources (web pages on FlashAttention; cited by page title and section):
+ *   [G]  "Flash Attention" glossary entry -- "How it works" (queries, keys and
+ *        values combined through normalised scores), "Worked example" (the
+ *        4,096 x 4,096 score matrix), "Common misconceptions" (exact does not
+ *        mean bit-identical).
+ *   [W]  "What Is FlashAttention? Why Long Context Got Cheap" -- "The problem it
+ *        solves" (the textbook method builds the n x n score matrix, applies
+ *        softmax, multiplies by V) and "What FlashAttention does instead"
+ *        (running max and running sum per row).
+ *   [L]  "How Flash Attention Improves Transformer Memory Efficiency Compared
+ *        to Standard Attention" -- "The Three Running Statistics" (the m, l and
+ *        unnormalised-output update rules and the final division), "Backward
+ *        Pass Efficiency" (statistics D_i, l_i, m_i), "Basic Flash Attention
+ *        Forward Pass" (shapes (B, H, L, D) and scale = 1/sqrt(D)).
+ *
+ * Conventions (readings where the pages are silent):
+ *   - Layout: every tensor is contiguous row-major [B, H, L, d].
+ *   - Scores are t_ij = scale * (q_i . k_j); the mask removes keys before the
+ *     softmax.  A key j is permitted for query row i when j < Lk and, under the
+ *     causal mask, j <= i + (Lk - Lq) (query i sits at absolute position
+ *     i + Lk - Lq, the reading that fits a cached prefix of keys).
+ *   - LSE_i = ln sum_j exp(t_ij) over the permitted keys (natural log, in units
+ *     of the scaled score).  A row with no permitted key has O_i = 0 and
+ *     LSE_i = -inf.
+ *   - Inputs may be given as doubles or as bfloat16 bit patterns (uint16); a
+ *     bfloat16 value converts to double exactly.
+ *
+ * Pinned by tests/test_oracle_pins.py against closed forms, limits, a brute
+ * force finite-difference gradient and the counts printed in [G] and [W].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_F64 0
+#define ORACLE_BF16 1
+
+/* bfloat16 is the upper half of an IEEE binary32; widening is exact. */
+static double bf16_bits_to_double(uint16_t h) {
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static double elem(const void* p, int64_t i, int dtype) {
+    if (dtype == ORACLE_BF16) return bf16_bits_to_double(((const uint16_t*)p)[i]);
+    return ((const double*)p)[i];
+}
+
+/* Number of permitted keys for query row i: keys 0 .. n-1 (the causal mask and
+ * the length bound both cut a prefix). */
+int64_t oracle_permitted_keys(int64_t i, int64_t Lq, int64_t Lk, int causal) {
+    int64_t n = Lk;
+    if (causal) {
+        int64_t last = i + (Lk - Lq);          /* highest permitted key index */
+        if (last + 1 < n) n = last + 1;
+    }
+    return n < 0 ? 0 : n;
+}
+
+/* Worked example of [G] and "The problem it solves" of [W]: the number of
+ * entries of the B x H x Lq x Lk score matrix the textbook method builds. */
+int64_t oracle_score_elements(int64_t B, int64_t H, int64_t Lq, int64_t Lk) {
+    return B * H * Lq * Lk;
+}
+
+/*
+ * One query row, two passes over its permitted keys ([W] "The problem it
+ * solves": scores, softmax over the whole row, weighted sum of V rows):
+ *   t_j = scale * q . k_j           for j < n
+ *   M   = max_j t_j
+ *   Z   = sum_j exp(t_j - M)
+ *   O   = sum_j (exp(t_j - M) / Z) v_j
+ *   LSE = M + ln Z
+ * t is caller scratch of length >= n (one score row, never an n x n matrix).
+ */
+static void attend_row(const void* q, int64_t q_off, const void* k, const void* v,
+                       int64_t kv_off, int64_t n, int64_t d, double scale, int dtype,
+                       double* t, double* o_row, double* lse_out) {
+    for (int64_t c = 0; c < d; ++c) o_row[c] = 0.0;
+    if (n <= 0) {
+        *lse_out = -INFINITY;
+        return;
+    }
+    double M = -INFINITY;
+    for (int64_t j = 0; j < n; ++j) {
+        double s = 0.0;
+        for (int64_t c = 0; c < d; ++c)
+            s += elem(q, q_off + c, dtype) * elem(k, kv_off + j * d + c, dtype);
+        t[j] = scale * s;
+        if (t[j] > M) M = t[j];
+    }
+    double Z = 0.0;
+    for (int64_t j = 0; j < n; ++j) Z += exp(t[j] - M);
+    for (int64_t j = 0; j < n; ++j) {
+        double p = exp(t[j] - M) / Z;
+        for (int64_t c = 0; c < d; ++c) o_row[c] += p * elem(v, kv_off + j * d + c, dtype);
+    }
+    *lse_out = M + log(Z);
+}
+
+/*
+ * Forward pass, all rows: O [B,H,Lq,d] and LSE [B,H,Lq] in double.
+ */
+void oracle_forward(const void* q, const void* k, const void* v, int dtype,
+                    double* o, double* lse, int64_t B, int64_t H, int64_t Lq,
+                    int64_t Lk, int64_t d, double scale, int causal) {
+    int64_t rows = B * H * Lq;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            int64_t bh = r / Lq, i = r % Lq;
+            int64_t n = oracle_permitted_keys(i, Lq, Lk, causal);
+            attend_row(q, r * d, k, v, bh * Lk * d, n, d, scale, dtype, t, o + r * d,
+                       lse + r);
+        }
+        free(t);
+    }
+}
+
+/*
+ * Forward pass on a chosen set of rows.  rows[s] is a flat row index
+ * (b*H + h)*Lq + i; the result for it goes to o_out[s*d ...] and lse_out[s].
+ * Row sampling is exact: each row of the output depends on that query row
+ * and all keys/values of its head only.
+ */
+void oracle_forward_rows(const void* q, const void* k, const void* v, int dtype,
+                         const int64_t* rows, int64_t n_rows, double* o_out,
+                         double* lse_out, int64_t B, int64_t H, int64_t Lq, int64_t Lk,
+                         int64_t d, double scale, int causal) {
+    (void)B;
+    (void)H;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t s = 0; s < n_rows; ++s) {
+            int64_t r = rows[s];
+            int64_t bh = r / Lq, i = r % Lq;
+            int64_t n = oracle_permitted_keys(i, Lq, Lk, causal);
+            attend_row(q, r * d, k, v, bh * Lk * d, n, d, scale, dtype, t,
+                       o_out + s * d, lse_out + s);
+        }
+        free(t);
+    }
+}
+
+/*
+ * The blockwise recurrence of [L] "The Three Running Statistics", taken
+ * literally on one row at a time: start from m = -inf, l = 0, O~ = 0; for each
+ * block of `block` keys,
+ *   m_new = max(m, max_j t_j)
+ *   l    <- exp(m - m_new) l + sum_j exp(t_j - m_new)
+ *   O~   <- exp(m - m_new) O~ + sum_j exp(t_j - m_new) v_j
+ *   m    <- m_new
+ * and finally O = O~ / l.  The running max is carried in scaled-score units.
+ * Used only to check that the recurrence reproduces the two-pass result.
+ */
+void oracle_forward_blockwise(const void* q, const void* k, const void* v, int dtype,
+                              double* o, double* lse, int64_t B, int64_t H, int64_t Lq,
+                              int64_t Lk, int64_t d, double scale, int causal,
+                              int64_t block) {
+    int64_t rows = B * H * Lq;
+    double* acc = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t bh = r / Lq, i = r % Lq;
+        int64_t n = oracle_permitted_keys(i, Lq, Lk, causal);
+        const int64_t kv_off = bh * Lk * d;
+        double m = -INFINITY, l = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc[c] = 0.0;
+        for (int64_t j0 = 0; j0 < n; j0 += block) {
+            int64_t j1 = j0 + block < n ? j0 + block : n;
+            double m_new = m;
+            for (int64_t j = j0; j < j1; ++j) {
+                double s = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    s += elem(q, r * d + c, dtype) * elem(k, kv_off + j * d + c, dtype);
+                if (scale * s > m_new) m_new = scale * s;
+            }
+            double alpha = (m == -INFINITY) ? 0.0 : exp(m - m_new);
+            l *= alpha;
+            for (int64_t c = 0; c < d; ++c) acc[c] *= alpha;
+            for (int64_t j = j0; j < j1; ++j) {
+                double s = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    s += elem(q, r * d + c, dtype) * elem(k, kv_off + j * d + c, dtype);
+                double p = exp(scale * s - m_new);
+                l += p;
+                for (int64_t c = 0; c < d; ++c) acc[c] += p * elem(v, kv_off + j * d + c, dtype);
+            }
+            m = m_new;
+        }
+        for (int64_t c = 0; c < d; ++c) o[r * d + c] = (n > 0) ? acc[c] / l : 0.0;
+        lse[r] = (n > 0) ? m + log(l) : -INFINITY;
+    }
+    free(acc);
+}
+
+/*
+ * Backward pass by differentiating the definition row by row ([L] "Backward
+ * Pass Efficiency" names the per-row statistic D_i; [G] "How it works" says the
+ * probabilities are recomputed rather than stored).  For each row i with its
+ * permitted keys j:
+ *   P_ij  = exp(t_ij - LSE_i)            (recomputed from the definition)
+ *   dP_ij = dO_i . v_j
+ *   D_i   = sum_j P_ij dP_ij             (equals dO_i . O_i)
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j += scale * dS_ij q_i
+ *   dV_j += P_ij dO_i
+ * Also returns D [B,H,Lq] when d_out is not NULL.  Parallel over heads only,
+ * since every row of a head adds into that head's dK and dV.
+ */
+void oracle_backward(const void* q, const void* k, const void* v, const void* dO,
+                     int dtype, double* dq, double* dk, double* dv, double* d_out,
+                     int64_t B, int64_t H, int64_t Lq, int64_t Lk, int64_t d,
+                     double scale, int causal) {
+    int64_t heads = B * H;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double* p = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double* dp = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            const int64_t kv_off = bh * Lk * d;
+            double* dk_h = dk + kv_off;
+            double* dv_h = dv + kv_off;
+            for (int64_t x = 0; x < Lk * d; ++x) {
+                dk_h[x] = 0.0;
+                dv_h[x] = 0.0;
+            }
+            for (int64_t i = 0; i < Lq; ++i) {
+                int64_t r = bh * Lq + i;
+                int64_t n = oracle_permitted_keys(i, Lq, Lk, causal);
+                double* dq_i = dq + r * d;
+                for (int64_t c = 0; c < d; ++c) dq_i[c] = 0.0;
+                if (n <= 0) {
+                    if (d_out) d_out[r] = 0.0;
+                    continue;
+                }
+                double M = -INFINITY;
+                for (int64_t j = 0; j < n; ++j) {
+                    double s = 0.0;
+                    for (int64_t c = 0; c < d; ++c)
+                        s += elem(q, r * d + c, dtype) * elem(k, kv_off + j * d + c, dtype);
+                    t[j] = scale * s;
+                    if (t[j] > M) M = t[j];
+                }
+                double Z = 0.0;
+                for (int64_t j = 0; j < n; ++j) Z += exp(t[j] - M);
+                double lse = M + log(Z);
+                double D = 0.0;
+                for (int64_t j = 0; j < n; ++j) {
+                    p[j] = exp(t[j] - lse);
+                    double s = 0.0;
+                    for (int64_t c = 0; c < d; ++c)
+                        s += elem(dO, r * d + c, dtype) * elem(v, kv_off + j * d + c, dtype);
+                    dp[j] = s;
+                    D += p[j] * dp[j];
+                }
+                if (d_out) d_out[r] = D;
+                for (int64_t j = 0; j < n; ++j) {
+                    double ds = p[j] * (dp[j] - D);
+                    for (int64_t c = 0; c < d; ++c) {
+                        dq_i[c] += scale * ds * elem(k, kv_off + j * d + c, dtype);
+                        dk_h[j * d + c] += scale * ds * elem(q, r * d + c, dtype);
+                        dv_h[j * d + c] += p[j] * elem(dO, r * d + c, dtype);
+                    }
+                }
+            }
+        }
+        free(t);
+        free(p);
+        free(dp);
+    }
+}
+
+/*
+ * Single-query decode over a key/value cache: for each (b, h), the forward
+ * pass with one query row and keys [0, kv_lens[b]) of a cache of capacity cap.
+ * q [B,H,d], caches [B,H,cap,d], o [B,H,d], lse [B,H].  kv_lens outside
+ * [0, cap] are clamped to that range.
+ */
+void oracle_decode(const void* q, const void* kcache, const void* vcache, int dtype,
+                   const int32_t* kv_lens, double* o, double* lse, int64_t B, int64_t H,
+                   int64_t cap, int64_t d, double scale) {
+    int64_t heads = B * H;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            int64_t n = kv_lens[bh / H];
+            if (n < 0) n = 0;
+            if (n > cap) n = cap;
+            attend_row(q, bh * d, kcache, vcache, bh * cap * d, n, d, scale, dtype, t,
+                       o + bh * d, lse + bh);
+        }
+        free(t);
+    }
+}
+
+/*
+ * Merge of partial results over disjoint key sets.  Given, for one row, parts
+ * s = 0..n-1 with normalised outputs O_s (d each) and LSE_s, the result over
+ * the union of the key sets is
+ *   LSE = ln sum_s exp(LSE_s)      O = sum_s exp(LSE_s - LSE) O_s .
+ * This is the recurrence of [L] "The Three Running Statistics" applied to whole
+ * blocks (m = LSE_s, l = 1, O~ = O_s for each part).  Parts with LSE_s = -inf
+ * (empty key sets) contribute nothing.
+ */
+void oracle_merge(const double* o_parts, const double* lse_parts, int64_t n, int64_t d,
+                  double* o, double* lse) {
+    double M = -INFINITY;
+    for (int64_t s = 0; s < n; ++s)
+        if (lse_parts[s] > M) M = lse_parts[s];
+    for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+    if (M == -INFINITY) {
+        *lse = -INFINITY;
+        return;
+    }
+    double Z = 0.0;
+    for (int64_t s = 0; s < n; ++s) Z += exp(lse_parts[s] - M);
+    double L = M + log(Z);
+    for (int64_t s = 0; s < n; ++s) {
+        double w = exp(lse_parts[s] - L);
+        for (int64_t c = 0; c < d; ++c) o[c] += w * o_parts[s * d + c];
+    }
+    *lse = L;
+}
+
+int oracle_num_threads(void) {
+    int n = 1;
+#pragma omp parallel
+    {
+#pragma omp single
+        {
+#ifdef _OPENMP
+            n = omp_get_num_threads();
+#endif
+        }
+    }
+    return n;
+}
