@@ -1,0 +1,217 @@
+// C ABI of the library (declared in include/fa.h): argument checks, TMA
+// descriptor encoding, launches, and the per-device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+__device__ int g_status;  // one per device; kernels record device-side conditions here
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool probed = false;
+    bool supported = false;
+    int num_sms = 0;
+    int* status_ptr = nullptr;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Resolves (once per device) whether the device is sm_100 and where its status word lives.
+int device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return FA_ERR_DEVICE;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.probed) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return FA_ERR_CUDA;
+        st.supported = (major == 10 && minor == 0);
+        if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return FA_ERR_CUDA;
+        if (st.supported) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return FA_ERR_CUDA;
+            st.status_ptr = static_cast<int*>(ptr);
+        }
+        st.probed = true;
+    }
+    if (!st.supported) return FA_ERR_DEVICE;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return FA_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    *out = &st;
+    return FA_OK;
+}
+
+// View a contiguous bf16 [BH, L, d] tensor as a 3-D TMA map with 128-row x
+// 64-column boxes and 128-byte swizzle (64 bf16 = one 128-byte swizzle span).
+// Rows past L read as zero; nothing outside the tensor is touched.
+int encode_rows_map(CUtensorMap* map, const void* base, int BH, int L, int d, int box_rows) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+bool dims_ok(int B, int H, int L, int d) {
+    if (B <= 0 || H <= 0 || L <= 0) return false;
+    const long long bh = static_cast<long long>(B) * H;
+    if (bh > (1LL << 30)) return false;
+    if (static_cast<long long>(L) * d * 2 >= (1LL << 40)) return false;
+    return true;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(int status) {
+    switch (status) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dimension or dtype";
+        case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA runtime error";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
+        case FA_ERR_DEVICE: return "FA_ERR_DEVICE: current device is not compute capability 10.0 (sm_100a)";
+        case FA_ERR_KV_LEN: return "FA_ERR_KV_LEN: a decode cache length was outside [0, cap]";
+        default: return "unknown fa_status";
+    }
+}
+
+int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,
+               int d, float scale, int causal, int o_dtype, void* stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
+    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_INVALID_ARG;
+    const long long n_ctas = static_cast<long long>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+    if (n_ctas > 0x7FFFFFFFLL) return FA_ERR_INVALID_ARG;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+
+    FwdParams p{};
+    const int BH = B * H;
+    if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, kFwdBM)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    p.o = o;
+    p.lse = lse;
+    p.status = st->status_ptr;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.o_dtype = o_dtype;
+    cudaError_t e = launch_fwd(p, d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int cap, int d) {
+    if (B <= 0 || H <= 0 || cap <= 0 || (d != 64 && d != 128)) return 0;
+    return decode_workspace_bytes(B, H, cap, d);
+}
+
+int fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens, void* o, float* lse,
+              int B, int H, int cap, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
+              void* stream) {
+    if (!q || !kcache || !vcache || !kv_lens || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (!dims_ok(B, H, cap, d) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
+        !aligned(kv_lens, 4) || !aligned(lse, 4))
+        return FA_ERR_INVALID_ARG;
+    const long long items = static_cast<long long>(B) * H * ((cap + kDecodeSplit - 1) / kDecodeSplit);
+    if (items > 0x7FFFFFFFLL || static_cast<long long>(B) * H > 0x7FFFFFFFLL) return FA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < decode_workspace_bytes(B, H, cap, d))
+        return FA_ERR_WORKSPACE;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+
+    DecodeParams p{};
+    p.q = q;
+    p.k = kcache;
+    p.v = vcache;
+    p.kv_lens = kv_lens;
+    p.o = o;
+    p.lse = lse;
+    p.status = st->status_ptr;
+    p.B = B;
+    p.H = H;
+    p.cap = cap;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_dtype = o_dtype;
+    decode_carve_workspace(p, workspace, B, H, cap, d);
+    cudaError_t e = launch_decode(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d) {
+    (void)B; (void)H; (void)Lq; (void)Lk; (void)d;
+    return 0;
+}
+
+int fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+    (void)q; (void)k; (void)v; (void)o; (void)dO; (void)lse; (void)dq; (void)dk; (void)dv; (void)B; (void)H;
+    (void)Lq; (void)Lk; (void)d; (void)scale; (void)causal; (void)o_dtype; (void)workspace;
+    (void)workspace_bytes; (void)stream;
+    return FA_ERR_UNSUPPORTED;
+}
+
+int fa_check_status(void* stream) {
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, st->status_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+    if (h != 0 && cudaMemset(st->status_ptr, 0, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    return h;
+}
+
+}  // extern "C"

@@ -1,0 +1,284 @@
+// Single-query decode over a KV cache, split over the key axis.
+//
+// The decode phase reads the whole cache once per generated token and does
+// about one FLOP per byte, so it is bound by HBM bandwidth ("What Is
+// FlashAttention?", "What it changes for you": the cache lives in HBM).  The
+// keys of each sequence are cut into fixed chunks of kDecodeSplit keys; every
+// chunk of every (b, h) is an independent work item that streams its K and V
+// rows with coalesced 128-bit loads, runs the running-max / running-sum
+// recurrence of "The Three Running Statistics" over them, and writes a
+// normalised partial output with its log-sum-exp.  A combine kernel merges the
+// partials of each (b, h) with the same recurrence applied to whole chunks.
+//
+// Kernels:
+//   fa_decode_plan     one CTA: clamps kv_lens to [0, cap] (flagging bad ones) and
+//                      prefix-sums the chunk counts per sequence.
+//   fa_decode_split    persistent CTAs over all (b, h, chunk) items.
+//   fa_decode_combine  one CTA per (b, h): log-sum-exp merge of its chunks.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "fa_internal.h"
+
+namespace fa {
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float ex2f_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Eight bf16 values packed in a uint4 -> float.
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+    f[0] = __uint_as_float(u.x << 16);
+    f[1] = __uint_as_float(u.x & 0xFFFF0000u);
+    f[2] = __uint_as_float(u.y << 16);
+    f[3] = __uint_as_float(u.y & 0xFFFF0000u);
+    f[4] = __uint_as_float(u.z << 16);
+    f[5] = __uint_as_float(u.z & 0xFFFF0000u);
+    f[6] = __uint_as_float(u.w << 16);
+    f[7] = __uint_as_float(u.w & 0xFFFF0000u);
+}
+
+__global__ void __launch_bounds__(kPlanThreads) fa_decode_plan(DecodeParams p) {
+    __shared__ int part[kPlanThreads];
+    const int t = threadIdx.x;
+    const int per = (p.B + kPlanThreads - 1) / kPlanThreads;
+    const int b0 = min(p.B, t * per), b1 = min(p.B, b0 + per);
+    int local = 0;
+    for (int b = b0; b < b1; ++b) {
+        int n = p.kv_lens[b];
+        if (n < 0 || n > p.cap) {
+            atomicCAS(p.status, 0, FA_ERR_KV_LEN);
+            n = n < 0 ? 0 : p.cap;
+        }
+        p.lens[b] = n;
+        local += (n + kDecodeSplit - 1) / kDecodeSplit;
+    }
+    part[t] = local;
+    __syncthreads();
+    // inclusive scan over the per-thread counts (Hillis-Steele)
+    for (int s = 1; s < kPlanThreads; s <<= 1) {
+        const int add = (t >= s) ? part[t - s] : 0;
+        __syncthreads();
+        part[t] += add;
+        __syncthreads();
+    }
+    int run = part[t] - local;  // exclusive prefix
+    for (int b = b0; b < b1; ++b) {
+        p.cum[b] = run;
+        run += (p.lens[b] + kDecodeSplit - 1) / kDecodeSplit;
+    }
+    if (t == kPlanThreads - 1) p.cum[p.B] = part[t];
+}
+
+// D/8 lanes hold one key row (8 bf16 each); a warp covers 256/D keys per load.
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads, 3) fa_decode_split(DecodeParams p) {
+    constexpr int kLanesPerKey = D / 8;
+    constexpr int kGroupsPerWarp = 32 / kLanesPerKey;
+    constexpr int kGroups = (kDecodeThreads / 32) * kGroupsPerWarp;  // key groups per CTA
+    constexpr int kUnroll = 4;
+    constexpr int kStep = kGroups * kUnroll;
+
+    __shared__ float red_m[kGroups];
+    __shared__ float red_l[kGroups];
+    __shared__ float red_acc[kGroups][D];
+    __shared__ int s_item[3];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;  // key group of this thread
+    const int e0 = (lane % kLanesPerKey) * 8;                  // first element of its slice
+    const float sl2 = p.scale_log2;
+    const int total = p.cum[p.B] * p.H;
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        if (threadIdx.x == 0) {
+            // item -> (b, h, chunk): items are ordered by b, then h, then chunk
+            int lo = 0, hi = p.B;  // find b with H*cum[b] <= item < H*cum[b+1]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (p.cum[mid] * p.H <= item) lo = mid; else hi = mid;
+            }
+            const int nb = p.cum[lo + 1] - p.cum[lo];
+            const int local = item - p.cum[lo] * p.H;
+            s_item[0] = lo;
+            s_item[1] = local / nb;
+            s_item[2] = local % nb;
+        }
+        __syncthreads();
+        const int b = s_item[0], h = s_item[1], chunk = s_item[2];
+        const int len = p.lens[b];
+        const int start = chunk * kDecodeSplit;
+        const int end = min(start + kDecodeSplit, len);
+        const size_t bh = static_cast<size_t>(b) * p.H + h;
+        const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k) + bh * p.cap * D + e0;
+        const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.v) + bh * p.cap * D + e0;
+
+        float qf[8];
+        unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) + bh * D + e0), qf);
+
+        float m = -INFINITY, l = 0.0f;
+        float acc[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
+
+        for (int base = start; base < end; base += kStep) {
+            uint4 kr[kUnroll], vr[kUnroll];
+            bool valid[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int key = base + u * kGroups + g;
+                valid[u] = key < end;
+                kr[u] = valid[u] ? ld_stream_u4(kbase + static_cast<size_t>(key) * D) : make_uint4(0, 0, 0, 0);
+                vr[u] = valid[u] ? ld_stream_u4(vbase + static_cast<size_t>(key) * D) : make_uint4(0, 0, 0, 0);
+            }
+            float s[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                float kf[8];
+                unpack8(kr[u], kf);
+                float dot = 0.0f;
+#pragma unroll
+                for (int x = 0; x < 8; ++x) dot = fmaf(qf[x], kf[x], dot);
+#pragma unroll
+                for (int o = kLanesPerKey / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                s[u] = valid[u] ? dot : -INFINITY;
+            }
+            float mb = s[0];
+#pragma unroll
+            for (int u = 1; u < kUnroll; ++u) mb = fmaxf(mb, s[u]);
+            const float m_new = fmaxf(m, mb);
+            // m_new is -inf only while this group has seen no valid key: then
+            // alpha = 0 and every p = 0, leaving l = 0 and acc = 0.
+            const float m_use = (m_new == -INFINITY) ? 0.0f : m_new;
+            const float alpha = (m == -INFINITY) ? 0.0f : ex2f_approx((m - m_use) * sl2);
+            const float mbias = m_use * sl2;
+            l *= alpha;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) acc[x] *= alpha;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const float pu = ex2f_approx(fmaf(s[u], sl2, -mbias));  // 0 for invalid keys
+                l += pu;
+                float vf[8];
+                unpack8(vr[u], vf);
+#pragma unroll
+                for (int x = 0; x < 8; ++x) acc[x] = fmaf(pu, vf[x], acc[x]);
+            }
+            m = m_new;
+        }
+
+        // merge the key groups of this CTA (same recurrence over whole groups)
+        if (lane % kLanesPerKey == 0) {
+            red_m[g] = m;
+            red_l[g] = l;
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) red_acc[g][e0 + x] = acc[x];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            const int c = threadIdx.x;
+            float M = -INFINITY;
+            for (int i = 0; i < kGroups; ++i) M = fmaxf(M, red_m[i]);
+            float L = 0.0f, O = 0.0f;
+            for (int i = 0; i < kGroups; ++i) {
+                if (red_m[i] == -INFINITY) continue;
+                const float w = ex2f_approx((red_m[i] - M) * sl2);
+                L = fmaf(w, red_l[i], L);
+                O = fmaf(w, red_acc[i][c], O);
+            }
+            const size_t slot = bh * p.max_splits + chunk;
+            p.part_o[slot * D + c] = O / L;
+            if (c == 0) p.part_lse[slot] = M * p.scale + logf(L);
+        }
+        __syncthreads();
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) fa_decode_combine(DecodeParams p) {
+    const int bh = blockIdx.x;
+    const int b = bh / p.H;
+    const int c = threadIdx.x;
+    const int n = (p.lens[b] + kDecodeSplit - 1) / kDecodeSplit;
+    const size_t out = static_cast<size_t>(bh) * D + c;
+    if (n == 0) {
+        if (p.o_dtype == FA_DT_F32) static_cast<float*>(p.o)[out] = 0.0f;
+        else static_cast<__nv_bfloat16*>(p.o)[out] = __float2bfloat16_rn(0.0f);
+        if (c == 0) p.lse[bh] = -INFINITY;
+        return;
+    }
+    const float* lse_s = p.part_lse + static_cast<size_t>(bh) * p.max_splits;
+    const float* o_s = p.part_o + static_cast<size_t>(bh) * p.max_splits * D;
+    float M = -INFINITY;
+    for (int s = 0; s < n; ++s) M = fmaxf(M, lse_s[s]);
+    float L = 0.0f, O = 0.0f;
+    for (int s = 0; s < n; ++s) {
+        const float w = __expf(lse_s[s] - M);
+        L += w;
+        O = fmaf(w, o_s[static_cast<size_t>(s) * D + c], O);
+    }
+    O /= L;
+    if (p.o_dtype == FA_DT_F32) static_cast<float*>(p.o)[out] = O;
+    else static_cast<__nv_bfloat16*>(p.o)[out] = __float2bfloat16_rn(O);
+    if (c == 0) p.lse[bh] = M + logf(L);
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int B, int H, int cap, int d) {
+    const size_t max_splits = (static_cast<size_t>(cap) + kDecodeSplit - 1) / kDecodeSplit;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t bh = static_cast<size_t>(B) * H;
+    return up(bh * max_splits * d * sizeof(float)) + up(bh * max_splits * sizeof(float)) +
+           up(static_cast<size_t>(B) * sizeof(int)) + up((static_cast<size_t>(B) + 1) * sizeof(int));
+}
+
+void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, int d) {
+    const size_t max_splits = (static_cast<size_t>(cap) + kDecodeSplit - 1) / kDecodeSplit;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t bh = static_cast<size_t>(B) * H;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    p.part_o = reinterpret_cast<float*>(w);
+    w += up(bh * max_splits * d * sizeof(float));
+    p.part_lse = reinterpret_cast<float*>(w);
+    w += up(bh * max_splits * sizeof(float));
+    p.lens = reinterpret_cast<int*>(w);
+    w += up(static_cast<size_t>(B) * sizeof(int));
+    p.cum = reinterpret_cast<int*>(w);
+    p.max_splits = static_cast<int>(max_splits);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream) {
+    fa_decode_plan<<<1, kPlanThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long upper = static_cast<long long>(p.B) * p.H * p.max_splits;
+    const int grid = static_cast<int>(std::min<long long>(upper, static_cast<long long>(num_sms) * 3));
+    if (d == 128) {
+        fa_decode_split<128><<<grid, kDecodeThreads, 0, stream>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        fa_decode_combine<128><<<p.B * p.H, 128, 0, stream>>>(p);
+    } else {
+        fa_decode_split<64><<<grid, kDecodeThreads, 0, stream>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        fa_decode_combine<64><<<p.B * p.H, 64, 0, stream>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fa

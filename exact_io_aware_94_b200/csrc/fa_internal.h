@@ -1,0 +1,67 @@
+// Internal declarations shared by the host API and the kernel translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa.h"
+
+namespace fa {
+
+// Every bounded wait in a kernel gives up after this long (nanoseconds of
+// %globaltimer), records FA_ERR_TIMEOUT and lets the CTA exit.
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+
+// Forward kernel tiling: two 128-row Q tiles per CTA (one per softmax
+// warpgroup), 128-key K/V tiles.
+constexpr int kFwdBM = 128;
+constexpr int kFwdBN = 128;
+constexpr int kFwdRowsPerCta = 2 * kFwdBM;
+constexpr int kFwdThreads = 320;  // 2 softmax warpgroups + TMA warp + MMA warp
+
+struct __align__(64) FwdParams {
+    CUtensorMap tm_q;  // [B*H, Lq, d] bf16, box {64, 128, 1}, 128B swizzle
+    CUtensorMap tm_k;  // [B*H, Lk, d]
+    CUtensorMap tm_v;  // [B*H, Lk, d]
+    void* o;
+    float* lse;
+    int* status;
+    int B, H, Lq, Lk;
+    float scale;       // multiplies q.k
+    float scale_log2;  // scale * log2(e)
+    int causal;
+    int o_dtype;
+};
+
+// Decode: keys of each sequence are cut into chunks of kDecodeSplit keys.
+constexpr int kDecodeSplit = 1024;
+constexpr int kDecodeThreads = 256;
+
+struct DecodeParams {
+    const void* q;        // [B, H, d] bf16
+    const void* k;        // [B, H, cap, d] bf16
+    const void* v;        // [B, H, cap, d] bf16
+    const int* kv_lens;   // [B]
+    void* o;              // [B, H, d]
+    float* lse;           // [B, H]
+    int* status;
+    // workspace
+    float* part_o;        // [B*H, max_splits, d] normalised partial outputs
+    float* part_lse;      // [B*H, max_splits]
+    int* lens;            // [B] clamped lengths
+    int* cum;             // [B+1] prefix sums of chunk counts
+    int B, H, cap, max_splits;
+    float scale, scale_log2;
+    int o_dtype;
+};
+
+size_t decode_workspace_bytes(int B, int H, int cap, int d);
+void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, int d);
+cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
+
+int fwd_smem_bytes(int d);
+cudaError_t launch_fwd(const FwdParams& p, int d, cudaStream_t stream);
+
+}  // namespace fa

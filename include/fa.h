@@ -1,0 +1,132 @@
+/*
+ * fa.h -- C ABI of the exact IO-aware attention library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T + mask) V
+ * tile by tile with the online-softmax recurrence (running max m_i, running
+ * sum l_i, unnormalised accumulator rescaled by exp(m_i - m_i_new), final
+ * division O_i = O~_i / l_i), so the L x L score and probability matrices never
+ * reach device memory.  Definitions follow the pages:
+ *   - "Flash Attention" glossary entry, "How it works": blocks of Q, K, V are
+ *     combined in on-chip memory with a running normalisation; the backward
+ *     pass recomputes intermediates instead of storing them.
+ *   - "What Is FlashAttention?", "What FlashAttention does instead": running
+ *     maximum and running sum per row; the score tile never reaches HBM.
+ *   - "How Flash Attention Improves Transformer Memory Efficiency ...",
+ *     "The Three Running Statistics" (the update rules above) and "Backward
+ *     Pass Efficiency" (per-row statistics D_i instead of stored matrices);
+ *     "Basic Flash Attention Forward Pass": q, k, v of shape (B, H, L, D),
+ *     scale = 1/sqrt(D), causal flag.
+ *
+ * Conventions shared by every call
+ *   Layout      Q, O, dO, dQ: contiguous row-major [B, H, Lq, d]; K, V, dK, dV:
+ *               [B, H, Lk, d]; LSE: fp32 [B, H, Lq]; decode caches [B, H, cap, d].
+ *   Types       Q, K, V, dO, caches: bfloat16.  O: bfloat16 or fp32 (o_dtype).
+ *               dQ, dK, dV: bfloat16.  Accumulation is fp32 throughout.
+ *   Mask        causal != 0 permits key j for query row i iff j <= i + (Lk - Lq)
+ *               (bottom-right alignment; identical to j <= i when Lq == Lk).
+ *               Causal calls require Lq <= Lk.
+ *   LSE         LSE_i = ln sum_j exp(scale * q_i . k_j) over permitted keys
+ *               (natural log, scaled-score units).
+ *   Pointers    All tensor pointers are DEVICE pointers on the current CUDA
+ *               device, 16-byte aligned.  The caller owns every buffer; the
+ *               library never allocates, frees or synchronises.  Calls are
+ *               asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   Devices     Compute capability 10.0 (sm_100a) only; elsewhere calls return
+ *               FA_ERR_DEVICE.  There is no fallback path.
+ *   Errors      Argument errors are returned synchronously and nothing is
+ *               launched.  A failed launch returns FA_ERR_CUDA.  Conditions met
+ *               on the device (a bounded wait that ran out, a cache length outside
+ *               [0, cap]) are recorded in a per-device status word read by
+ *               fa_check_status().  No kernel traps.
+ */
+#ifndef EXACT_IO_AWARE_FA_H
+#define EXACT_IO_AWARE_FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, misalignment, causal with Lq > Lk */
+    FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, dtype code unknown */
+    FA_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than *_workspace_size() */
+    FA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+    FA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
+    FA_ERR_DEVICE = 6,      /* current device is not compute capability 10.0 */
+    FA_ERR_KV_LEN = 7       /* device: a decode cache length was outside [0, cap] (clamped) */
+} fa_status;
+
+enum { FA_DT_BF16 = 0, FA_DT_F32 = 1 };
+
+/*
+ * Forward pass ("How it works" of the glossary entry; "The Three Running
+ * Statistics").  Reads q [B,H,Lq,d], k and v [B,H,Lk,d] (bf16); writes
+ * o [B,H,Lq,d] (bf16 if o_dtype == FA_DT_BF16, fp32 if FA_DT_F32) and
+ * lse [B,H,Lq] (fp32).  scale multiplies q.k before the softmax (typically
+ * 1/sqrt(d)).  d must be 64 or 128.  Rows never see keys beyond Lk; nothing
+ * past the end of any tensor is read.
+ */
+int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,
+               int d, float scale, int causal, int o_dtype, void* stream);
+
+/*
+ * Workspace bytes fa_backward needs for these sizes: the per-row statistic
+ * D [B,H,Lq] (fp32) and an fp32 dQ accumulator [B,H,Lq,d], each 256-byte
+ * aligned.  Returns 0 for invalid sizes.
+ */
+size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d);
+
+/*
+ * Backward pass with recomputation ("Backward Pass Efficiency"; glossary "How
+ * it works").  Inputs: q, k, v, the forward output o (o_dtype) and its
+ * lse, and the output gradient dO [B,H,Lq,d] (bf16).  Outputs dq [B,H,Lq,d],
+ * dk and dv [B,H,Lk,d] (bf16).  P is recomputed from lse; no L x L matrix is
+ * stored.  workspace: device memory of at least fa_backward_workspace_size()
+ * bytes, 256-byte aligned, owned by the caller; its contents on entry do not
+ * matter and on return are unspecified.
+ */
+int fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                int o_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes fa_decode needs: split-KV partial results (fp32 output
+ * vector and LSE per split) for B*H heads and up to ceil(cap / split) splits.
+ */
+size_t fa_decode_workspace_size(int B, int H, int cap, int d);
+
+/*
+ * Single-query decode over a KV cache (the decode phase of "What Is
+ * FlashAttention?", "What it changes for you": the cache lives in HBM and is
+ * read once).  q [B,H,d] (bf16); kcache, vcache [B,H,cap,d] (bf16); kv_lens
+ * int32 [B] on the device, the number of valid cache rows of each sequence.
+ * Writes o [B,H,d] (o_dtype) and lse [B,H] (fp32).  Keys [0, kv_lens[b]) are
+ * split into fixed-size chunks processed in parallel; their partial
+ * (O, LSE) pairs are merged by a log-sum-exp combine.  A length outside
+ * [0, cap] is clamped and flagged as FA_ERR_KV_LEN in the status word; a
+ * length of 0 gives o = 0 and lse = -inf.  Slots at or past kv_lens[b] are
+ * never read.
+ */
+int fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens, void* o, float* lse,
+              int B, int H, int cap, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
+              void* stream);
+
+/*
+ * Synchronises `stream`, returns the current device's status word (FA_OK if no
+ * kernel recorded a condition since the last call) and clears it.  Returns
+ * FA_ERR_CUDA if the synchronisation itself fails.
+ */
+int fa_check_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_IO_AWARE_FA_H */
