@@ -1,0 +1,476 @@
+"""Benchmark of the exact-attention library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--legs all|none]
+
+Prints ONE JSON line (rank 0).  The headline workload is the forward pass at
+the pages' 4,096-token example: B=4, H=16, L=4096, d=128, causal, Q ~ 4 N(0,1)
+(peaky rows), bf16 inputs, fp32 O + LSE.  A step is one fa_forward over that
+batch; `value` is algorithmic TFLOP/s (4 B H L^2 d, halved for causal) of all
+ranks' work divided by the slowest rank's time.  The other measured paths of
+the library -- the training forward+backward at L=8192, the 65,536-token
+forward and the split-KV decode -- are reported under "legs", each with its
+own roofline.
+
+Multi-GPU: the path does not shard (each GPU is an independent replica); the
+ranks only share a barrier and a max-over-ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+HEADLINE = "fwd_L4096_peaky"
+METRIC = "attention fwd/bwd TFLOP/s and % of bf16 tensor peak; decode HBM GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16, datasheet
+NOMINAL_HBM_GBS = 8000.0
+
+
+# ----------------------------------------------------------------------------- host helpers
+def attn_flops(B, H, Lq, Lk, d, causal, backward=False):
+    f = 4.0 * B * H * Lq * Lk * d
+    if causal:
+        f *= 0.5
+    if backward:
+        f *= 2.5
+    return f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            m = json.load(fh)
+        return {k: float(m[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "exact_io_aware_94_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, src_files):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as fh:
+            rec = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    e = rec.get(kernel, {}).get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash(src_files):
+        return None
+    return e.get("bytes_per_launch")
+
+
+def reduce_max(value, dist=None, device=None):
+    """Max over ranks of a float (the slowest rank's time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(value, dist=None, device=None):
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.QUERY, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.25)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+        return False
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = []
+        mx = None
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in self.rows:
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU baseline (oracle)
+def oracle_forward_sample(workload, budget_s, seed=0):
+    """Time the oracle on a bounded sample of the forward workload's rows.
+
+    Returns (tflops, seconds, threads, description).  Each sampled row is a
+    complete output row (exact: rows are independent)."""
+    import numpy as np
+
+    import oracle
+    from exact_io_aware_94_b200.inputs import WORKLOADS, attention_inputs
+
+    w = WORKLOADS[workload]
+    B, H, L, d, causal = w["B"], w["H"], w["L"], w["d"], w["causal"]
+    # one head's inputs suffice for a row sample; same shapes and value distribution
+    inp = attention_inputs(1, 1, L, L, d, seed=w["seed"], q_scale=w["q_scale"])
+    rng = np.random.default_rng(seed)
+    scale = 1.0 / math.sqrt(d)
+
+    def run(n):
+        rows = rng.integers(0, L, size=n)
+        flops = sum(4.0 * d * oracle.permitted_keys(int(i), L, L, causal) for i in rows)
+        t0 = time.perf_counter()
+        oracle.forward_rows(inp.q, inp.k, inp.v, rows, scale, causal)
+        return flops, time.perf_counter() - t0
+
+    n = 64
+    f, t = run(n)
+    while t < budget_s / 8 and n < 1 << 20:
+        n *= 2
+        f, t = run(n)
+    if t < budget_s / 2:
+        n = max(n, int(n * (budget_s / 2) / max(t, 1e-6)))
+        f, t = run(n)
+    desc = "%d random query rows of one head of %s (B=%d H=%d L=%d d=%d causal=%s), %.1f s" % (
+        n, workload, B, H, L, d, causal, t)
+    return f / t / 1e12, t, oracle.num_threads(), desc
+
+
+# ----------------------------------------------------------------------------- GPU timing
+def time_steps(fn, steps, warmup, stream, dist=None, device=None):
+    """Warm up, then time exactly `steps` calls between barrier+synchronize pairs with
+    CUDA events on the launching stream; returns the max-over-ranks total seconds."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if dist is not None and dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None and dist.is_initialized():
+        dist.barrier()
+    torch.cuda.synchronize()
+    return reduce_max(start.elapsed_time(end) / 1e3, dist, device)
+
+
+def run_ours(args, dist, rank, world, device):
+    import torch
+
+    import exact_io_aware_94_b200 as fa
+    from exact_io_aware_94_b200.inputs import WORKLOADS
+
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream(device)
+    w = WORKLOADS[HEADLINE]
+    B, H, L, d, causal = w["B"], w["H"], w["L"], w["d"], w["causal"]
+    gen = torch.Generator(device=device).manual_seed(w["seed"] + 1000 * rank)
+    # seeded synthetic inputs of the workload's shape and distribution, resident in HBM
+    q = (torch.randn(B, H, L, d, generator=gen, device=device) * w["q_scale"]).to(torch.bfloat16)
+    k = torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16)
+    v = torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16)
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=device)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=device)
+    scale = 1.0 / math.sqrt(d)
+
+    def step():
+        rc = fa.fa_forward(q, k, v, o, lse, B, H, L, L, d, scale, causal, fa.FA_DT_F32, stream)
+        if rc != fa.FA_OK:
+            raise fa.FAError(rc, "fa_forward")
+
+    flops = attn_flops(B, H, L, L, d, causal)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        secs = time_steps(step, args.steps, args.warmup, stream, dist, device)
+    status = fa.fa_check_status(stream)
+    if status != fa.FA_OK:
+        raise fa.FAError(status, "device status after the timed region")
+    ms_per_step = secs / args.steps * 1e3
+    value = reduce_sum(flops * args.steps, dist, device) / secs / 1e12
+    achieved = flops / (secs / args.steps) / 1e12  # the step is one launch of the forward kernel
+    roof = {"kernel": "fa_fwd_kernel<128>", "bound": "tensor", "achieved": round(achieved, 1),
+            "peak": peaks["bf16_tflops"], "peak_kind": peak_kind + " burst bf16 (cuBLAS 8192^3)",
+            "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
+            "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+            "traffic": recorded_traffic("fa_fwd_kernel", HEADLINE, ["fwd_sm100.cu", "ptx.cuh"]),
+            "algorithmic_flops_per_launch": flops}
+
+    # ---- end to end through the public API: pinned host inputs in, O and LSE back to host, every step
+    qh = q.cpu().pin_memory()
+    kh = k.cpu().pin_memory()
+    vh = v.cpu().pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 10))
+    e2e_secs = time_steps(e2e_step, e2e_steps, max(1, args.warmup), stream, dist, device)
+    e2e_value = reduce_sum(flops * e2e_steps, dist, device) / e2e_secs / 1e12
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    legs = {}
+    launches = args.steps  # fa_forward launches exactly one kernel per call
+    if args.legs == "all":
+        del qh, kh, vh, oh, lh
+        legs = run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) bf16, Q x4), generated on device",
+        "config": {"workload": HEADLINE + ": forward, B=4 H=16 Lq=Lk=4096 d=128 causal, Q~4N(0,1), O fp32 + LSE",
+                   "global_batch": B * world, "seq_len": L, "parallelism": "replicas%d" % world,
+                   "l2": "inputs larger than L2 (192 MiB of Q/K/V per replica vs 126 MB L2)"},
+        "roofline": roof,
+        "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "path": "pinned host Q/K/V -> device, fa_forward, O/LSE -> pinned host"},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+        "legs": legs,
+    }
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        tf, secs_cpu, cores, desc = oracle_forward_sample(HEADLINE, args.cpu_budget)
+        out["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    return out
+
+
+def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
+    from exact_io_aware_94_b200.inputs import WORKLOADS
+
+    legs = {}
+    steps = max(3, min(args.steps, 20))
+    warm = max(3, args.warmup)
+
+    # training forward + backward at L = 8192
+    w = WORKLOADS["train_L8192"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    gen = torch.Generator(device=device).manual_seed(w["seed"] + 1000 * rank)
+    q, k, v, g = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(4))
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=device)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), device)
+    scale = 1.0 / math.sqrt(d)
+
+    def fwd():
+        rc = fa.fa_forward(q, k, v, o, lse, B, H, L, L, d, scale, 1, fa.FA_DT_F32, stream)
+        assert rc == fa.FA_OK
+
+    def bwd():
+        rc = fa.fa_backward(q, k, v, o, g, lse, dq, dk, dv, B, H, L, L, d, scale, 1, fa.FA_DT_F32, ws,
+                            ws.numel(), stream)
+        assert rc == fa.FA_OK
+
+    ff = attn_flops(B, H, L, L, d, True)
+    fb = attn_flops(B, H, L, L, d, True, backward=True)
+    t_f = time_steps(fwd, steps, warm, stream, dist, device) / steps
+    t_b = time_steps(bwd, steps, warm, stream, dist, device) / steps
+    legs["train_L8192_fwd"] = {"ms": round(t_f * 1e3, 4), "TFLOP/s": round(ff / t_f / 1e12, 1),
+                               "frac_of_peak": round(ff / t_f / 1e12 / peaks["bf16_tflops"], 4), "launches": 1}
+    legs["train_L8192_bwd"] = {"ms": round(t_b * 1e3, 4), "TFLOP/s": round(fb / t_b / 1e12, 1),
+                               "frac_of_peak": round(fb / t_b / 1e12 / peaks["bf16_tflops"], 4),
+                               "launches": 3, "kernels": "fa_bwd_dot + fa_bwd_dkdv + fa_bwd_dq",
+                               "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 7"}
+    del q, k, v, g, o, lse, dq, dk, dv, ws
+
+    # 65,536-token forward
+    w = WORKLOADS["long_L65536"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=device)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=device)
+
+    def fwd_long():
+        rc = fa.fa_forward(q, k, v, o, lse, B, H, L, L, d, scale, 1, fa.FA_DT_F32, stream)
+        assert rc == fa.FA_OK
+
+    fl = attn_flops(B, H, L, L, d, True)
+    t_l = time_steps(fwd_long, max(3, steps // 4), 3, stream, dist, device) / max(3, steps // 4)
+    legs["long_L65536_fwd"] = {"ms": round(t_l * 1e3, 4), "TFLOP/s": round(fl / t_l / 1e12, 1),
+                               "frac_of_peak": round(fl / t_l / 1e12 / peaks["bf16_tflops"], 4), "launches": 1}
+    del q, k, v, o, lse
+
+    # decode over a 32,768-slot cache
+    w = WORKLOADS["decode_cap32768"]
+    B, H, cap, d = w["B"], w["H"], w["cap"], w["d"]
+    cg = torch.Generator("cpu").manual_seed(w["seed"])
+    lens = torch.randint(w["len_lo"], w["len_hi"] + 1, (B,), generator=cg).to(torch.int32)
+    kc = torch.randn(B, H, cap, d, generator=gen, device=device).to(torch.bfloat16)
+    vc = torch.randn(B, H, cap, d, generator=gen, device=device).to(torch.bfloat16)
+    qd = torch.randn(B, H, d, generator=gen, device=device).to(torch.bfloat16)
+    lens_d = lens.to(device)
+    od = torch.empty(B, H, d, dtype=torch.float32, device=device)
+    ld = torch.empty(B, H, dtype=torch.float32, device=device)
+    wsd = fa.workspace(fa.fa_decode_workspace_size(B, H, cap, d), device)
+
+    def dec():
+        rc = fa.fa_decode(qd, kc, vc, lens_d, od, ld, B, H, cap, d, scale, fa.FA_DT_F32, wsd, wsd.numel(), stream)
+        assert rc == fa.FA_OK
+
+    nbytes = int(lens.sum()) * H * d * 2 * 2
+    t_d = time_steps(dec, steps, warm, stream, dist, device) / steps
+    legs["decode_cap32768"] = {"ms": round(t_d * 1e3, 4), "GB/s": round(nbytes / t_d / 1e9, 1),
+                               "kv_bytes": nbytes,
+                               "frac_of_peak": round(nbytes / t_d / 1e9 / peaks["hbm_gbs"], 4),
+                               "frac_of_nominal_8000": round(nbytes / t_d / 1e9 / NOMINAL_HBM_GBS, 4),
+                               "launches": 3, "kernels": "fa_decode_plan + fa_decode_split + fa_decode_combine",
+                               "l2": "caches 2 x 16 GiB, far larger than L2"}
+    del kc, vc
+    status = fa.fa_check_status(stream)
+    if status != fa.FA_OK:
+        raise fa.FAError(status, "device status after the legs")
+    return legs
+
+
+def run_reference(args, rank):
+    """The oracle, as it stands, on the host cores: bounded samples of the same workload."""
+    if rank != 0:
+        return None
+    vals = []
+    secs = []
+    desc = ""
+    cores = 0
+    for _ in range(args.warmup):
+        oracle_forward_sample(HEADLINE, 1.0)
+    for _ in range(args.steps):
+        tf, s, cores, desc = oracle_forward_sample(HEADLINE, args.ref_budget)
+        vals.append(tf)
+        secs.append(s)
+    value = statistics.median(vals)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.median(secs), 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) bf16, Q x4)",
+        "config": {"workload": HEADLINE + ": forward, B=4 H=16 Lq=Lk=4096 d=128 causal, Q~4N(0,1)",
+                   "global_batch": 4, "seq_len": 4096, "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--legs", choices=["all", "none"], default="all")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work per reference step")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    try:
+        out = run_ours(args, dist if world > 1 else None, rank, world, device)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

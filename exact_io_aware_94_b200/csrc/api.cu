@@ -189,17 +189,57 @@ int fa_decode(const void* q, const void* kcache, const void* vcache, const int* 
 }
 
 size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d) {
-    (void)B; (void)H; (void)Lq; (void)Lk; (void)d;
-    return 0;
+    if (B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || (d != 64 && d != 128)) return 0;
+    return bwd_workspace_bytes(B, H, Lq);
 }
 
 int fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                 void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
                 int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-    (void)q; (void)k; (void)v; (void)o; (void)dO; (void)lse; (void)dq; (void)dk; (void)dv; (void)B; (void)H;
-    (void)Lq; (void)Lk; (void)d; (void)scale; (void)causal; (void)o_dtype; (void)workspace;
-    (void)workspace_bytes; (void)stream;
-    return FA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
+    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+        return FA_ERR_INVALID_ARG;
+    const long long bh = static_cast<long long>(B) * H;
+    if (bh * ((Lq + 127) / 128) > 0x7FFFFFFFLL || bh * ((Lk + 127) / 128) > 0x7FFFFFFFLL ||
+        bh * Lq * (d / 8) / 256 > 0x7FFFFFFFLL)
+        return FA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < bwd_workspace_bytes(B, H, Lq))
+        return FA_ERR_WORKSPACE;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+
+    BwdParams p{};
+    const int BH = B * H;
+    if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_do, dO, BH, Lq, d, 128)) != FA_OK) return rc;
+    p.o = o;
+    p.dO = dO;
+    p.lse = lse;
+    p.dsum = static_cast<float*>(workspace);
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.status = st->status_ptr;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.o_dtype = o_dtype;
+    cudaError_t e = launch_bwd(p, d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_check_status(void* stream) {

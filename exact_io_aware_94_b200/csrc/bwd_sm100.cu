@@ -1,0 +1,655 @@
+// Backward pass of exact attention for sm_100a, by recomputation.
+//
+// The pages keep only per-row statistics for the backward pass and recompute
+// the probabilities instead of storing them ("Backward Pass Efficiency": D_i,
+// l_i, m_i; glossary "How it works": intermediates are recomputed).  Here the
+// saved statistic is LSE_i = m_i + ln l_i, so P_ij = exp(scale q_i.k_j - LSE_i).
+// With dP = dO V^T, D_i = rowsum(dO o O), dS = P o (dP - D):
+//     dV = P^T dO,   dK = scale dS^T Q,   dQ = scale dS K.
+//
+// Three kernels, no atomics (deterministic):
+//   fa_bwd_dot   D_i = sum_c dO_ic O_ic                        (HBM-bound)
+//   fa_bwd_dkdv  one CTA per (b, h, 128-key tile), loop over 128-row Q tiles:
+//                S^T = K Q^T and dP^T = V dO^T (SS MMA into TMEM); one thread
+//                per key row turns them into P^T and dS^T (bf16, written back
+//                into TMEM); dV += P^T dO and dK += dS^T Q (TS MMA, A from TMEM).
+//   fa_bwd_dq    one CTA per (b, h, 128-row Q tile), loop over 128-key tiles:
+//                S = Q K^T (double-buffered) and dP = dO V^T; one thread per
+//                query row forms dS (bf16, into TMEM); dQ += dS K (TS MMA).
+// Each of the two heavy kernels has two elementwise warpgroups that split the
+// 128 columns of every tile between them, a TMA producer warp and an MMA warp.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "fa_internal.h"
+#include "ptx.cuh"
+
+namespace fa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct BwdTiles {
+    static constexpr int kBoxBytes = 128 * 64 * 2;
+    static constexpr int kBoxes = D / 64;
+    static constexpr int kTileBytes = kBoxBytes * kBoxes;  // one 128-row bf16 tile
+    static constexpr int kStages = (D == 128) ? 2 : 4;
+};
+
+// ---------------------------------------------------------------- D = rowsum(dO o O)
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dot(BwdParams p) {
+    constexpr int kLanes = D / 8;  // lanes per row, 8 elements each
+    const long long rows = static_cast<long long>(p.B) * p.H * p.Lq;
+    const long long row = (static_cast<long long>(blockIdx.x) * 256 + threadIdx.x) / kLanes;
+    const int e0 = (threadIdx.x % kLanes) * 8;
+    float acc = 0.0f;
+    if (row < rows) {
+        const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.dO) + row * D + e0);
+        const float gf[8] = {__uint_as_float(g.x << 16), __uint_as_float(g.x & 0xFFFF0000u),
+                             __uint_as_float(g.y << 16), __uint_as_float(g.y & 0xFFFF0000u),
+                             __uint_as_float(g.z << 16), __uint_as_float(g.z & 0xFFFF0000u),
+                             __uint_as_float(g.w << 16), __uint_as_float(g.w & 0xFFFF0000u)};
+        if (p.o_dtype == FA_DT_F32) {
+            const float4* o = reinterpret_cast<const float4*>(static_cast<const float*>(p.o) + row * D + e0);
+            const float4 a = o[0], b = o[1];
+            acc = gf[0] * a.x + gf[1] * a.y + gf[2] * a.z + gf[3] * a.w + gf[4] * b.x + gf[5] * b.y +
+                  gf[6] * b.z + gf[7] * b.w;
+        } else {
+            const uint4 o = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.o) + row * D + e0);
+            acc = gf[0] * __uint_as_float(o.x << 16) + gf[1] * __uint_as_float(o.x & 0xFFFF0000u) +
+                  gf[2] * __uint_as_float(o.y << 16) + gf[3] * __uint_as_float(o.y & 0xFFFF0000u) +
+                  gf[4] * __uint_as_float(o.z << 16) + gf[5] * __uint_as_float(o.z & 0xFFFF0000u) +
+                  gf[6] * __uint_as_float(o.w << 16) + gf[7] * __uint_as_float(o.w & 0xFFFF0000u);
+        }
+    }
+#pragma unroll
+    for (int o = kLanes / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (row < rows && (threadIdx.x % kLanes) == 0) p.dsum[row] = acc;
+}
+
+// ---------------------------------------------------------------- dK, dV
+template <int D>
+struct DkdvLayout {
+    using T = BwdTiles<D>;
+    static constexpr int S = T::kStages;
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + T::kTileBytes;
+    static constexpr int kQOff = kVOff + T::kTileBytes;             // S stages
+    static constexpr int kGOff = kQOff + S * T::kTileBytes;         // dO, S stages
+    static constexpr int kStatOff = kGOff + S * T::kTileBytes;      // per stage: lse2[128], dsum[128]
+    static constexpr int kBarOff = kStatOff + S * 2 * 128 * 4;
+    // bars: kv, qd[S], empty[S], s, dp, p, ds, acc, drain
+    static constexpr int kNumBars = 1 + 2 * S + 6;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kBytes = kMiscOff + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1) fa_bwd_dkdv(const __grid_constant__ BwdParams p) {
+    using T = BwdTiles<D>;
+    using Lay = DkdvLayout<D>;
+    constexpr int S = Lay::S;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sK = smem + Lay::kKOff;
+    uint8_t* sV = smem + Lay::kVOff;
+    uint8_t* sQ = smem + Lay::kQOff;
+    uint8_t* sG = smem + Lay::kGOff;
+    float* sStat = reinterpret_cast<float*>(smem + Lay::kStatOff);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
+    uint64_t* bar_kv = bars;
+    uint64_t* bar_qd = bars + 1;
+    uint64_t* bar_empty = bars + 1 + S;
+    uint64_t* bar_s = bars + 1 + 2 * S;
+    uint64_t* bar_dp = bar_s + 1;
+    uint64_t* bar_p = bar_s + 2;
+    uint64_t* bar_ds = bar_s + 3;
+    uint64_t* bar_acc = bar_s + 4;
+    uint64_t* bar_drain = bar_s + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.B * p.H;
+    const int kt = static_cast<int>(blockIdx.x) / BH;  // small key tiles first: they see the most queries
+    const int bh = static_cast<int>(blockIdx.x) % BH;
+    const int j0 = kt * 128;
+    const int off = p.Lk - p.Lq;
+    const int nq_all = (p.Lq + 127) / 128;
+    const int qt0 = p.causal ? max(0, j0 - off) / 128 : 0;
+    const int nq = nq_all - qt0;  // >= 1: the last query row sees every key
+
+    // TMEM columns: S^T [0,128) dP^T [128,256) dV [256,256+D) dK [256+D,256+2D)
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_kv, 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bar_qd[s], 1 + 32);
+            mbar_init(&bar_empty[s], 1);
+        }
+        mbar_init(bar_s, 1);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_p, 256);
+        mbar_init(bar_ds, 256);
+        mbar_init(bar_acc, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = (atomicAdd(p.status, 0) == FA_ERR_TIMEOUT) ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 8) {
+        // ================= producer: K, V once; then Q, dO, LSE, D per query tile
+        int issued = 0;
+        if (!*abort_flag) {
+            if (lane == 0) {
+                tma_prefetch_desc(&p.tm_q);
+                tma_prefetch_desc(&p.tm_do);
+                mbar_arrive_expect_tx(bar_kv, 2 * T::kTileBytes);
+                for (int b = 0; b < T::kBoxes; ++b) {
+                    tma_load_3d(sK + b * T::kBoxBytes, &p.tm_k, bar_kv, b * 64, j0, bh);
+                    tma_load_3d(sV + b * T::kBoxBytes, &p.tm_v, bar_kv, b * 64, j0, bh);
+                }
+            }
+            for (int t = 0; t < nq; ++t) {
+                const int s = t % S;
+                bool ok = true;
+                if (t >= S) ok = mbar_wait(&bar_empty[s], ((t / S) - 1) & 1, abort_flag, p.status);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                const int i0 = (qt0 + t) * 128;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bar_qd[s], 2 * T::kTileBytes);
+                    for (int b = 0; b < T::kBoxes; ++b) {
+                        tma_load_3d(sQ + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_q, &bar_qd[s], b * 64, i0, bh);
+                        tma_load_3d(sG + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_do, &bar_qd[s], b * 64, i0, bh);
+                    }
+                }
+                float* st = sStat + s * 256;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int r = lane * 4 + x;
+                    const int i = i0 + r;
+                    const bool valid = i < p.Lq;
+                    const size_t idx = static_cast<size_t>(bh) * p.Lq + i;
+                    st[r] = valid ? p.lse[idx] * kLog2e : INFINITY;  // P = 0 for rows past Lq
+                    st[128 + r] = valid ? p.dsum[idx] : 0.0f;
+                }
+                mbar_arrive(&bar_qd[s]);
+                issued = t + 1;
+            }
+        }
+        if (lane == 0 && *abort_flag) {
+            mbar_wait_drain(bar_kv, 0, p.status);
+            for (int t = max(0, issued - S); t < issued; ++t) mbar_wait_drain(&bar_qd[t % S], (t / S) & 1, p.status);
+        }
+    } else if (warp == 9) {
+        // ================= MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sGa = smem_u32(sG);
+            bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status);
+            for (int t = 0; ok && t < nq; ++t) {
+                const int s = t % S;
+                if (!(ok = mbar_wait(&bar_qd[s], (t / S) & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+                // S^T = K Q^T, dP^T = V dO^T   (M = 128 keys, N = 128 queries, K = D)
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+                    umma_ss(tmem_base + kColS, smem_desc_sw128(sKa + koff, 16, 1024),
+                            smem_desc_sw128(sQa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                }
+                umma_commit(bar_s);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+                    umma_ss(tmem_base + kColDP, smem_desc_sw128(sVa + koff, 16, 1024),
+                            smem_desc_sw128(sGa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                }
+                umma_commit(bar_dp);
+                // dV += P^T dO   (A = P^T from TMEM: queries 0-63 at cols [0,32), 64-127 at [64,96))
+                if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = tmem_base + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem_base + kColDV, a,
+                            smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                // dK += dS^T Q
+                if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = tmem_base + kColDP + (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem_base + kColDK, a,
+                            smem_desc_sw128(sQa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                            (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bar_empty[s]);
+            }
+            if (ok) umma_commit(bar_acc);
+            umma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0, p.status);
+        }
+    } else {
+        // ================= elementwise: thread = key row, warpgroup w = query columns [64w, 64w+64)
+        const int w = warp >> 2, wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int key = j0 + r;
+        const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+        const uint32_t tS = tmem_base + lane_bits + kColS + w * 64;
+        const uint32_t tDP = tmem_base + lane_bits + kColDP + w * 64;
+        const float sl2 = p.scale_log2;
+        bool ok = true;
+        for (int t = 0; t < nq; ++t) {
+            const int s = t % S;
+            const int i0 = (qt0 + t) * 128 + w * 64;  // first query of this warpgroup's columns
+            const float* lse2 = sStat + s * 256 + w * 64;
+            const float* dsum = sStat + s * 256 + 128 + w * 64;
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_s, t & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            float pr[64];
+            {
+                uint32_t u[32];
+                tmem_ld32(tS, u);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) pr[x] = __uint_as_float(u[x]);
+                tmem_ld32(tS + 32, u);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) pr[32 + x] = __uint_as_float(u[x]);
+                tmem_wait_ld();
+            }
+            // P^T = exp2(S^T * scale*log2e - LSE*log2e); causal: key > query + off -> 0
+            const bool need_mask = p.causal && (j0 + 127 > i0 + off);
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float v = ex2_approx(fmaf(pr[c], sl2, -lse2[c]));
+                if (need_mask && key > i0 + c + off) v = 0.0f;
+                pr[c] = v;
+            }
+            {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_p);
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                uint32_t u[32], pk[32];
+                tmem_ld32(tDP, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(pr[2 * c] * (__uint_as_float(u[2 * c]) - dsum[2 * c]),
+                                        pr[2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum[2 * c + 1]));
+                tmem_ld32(tDP + 32, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[16 + c] = pack_bf16x2(pr[32 + 2 * c] * (__uint_as_float(u[2 * c]) - dsum[32 + 2 * c]),
+                                             pr[32 + 2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum[32 + 2 * c + 1]));
+                tmem_st32(tDP, pk);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_ds);
+        }
+        // epilogue: dV = acc, dK = scale * acc; warpgroup w writes columns [w*D/2, (w+1)*D/2)
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, 0, abort_flag, p.status));
+        if (ok) {
+            tc_fence_after();
+            const bool valid = key < p.Lk;
+            const size_t rowoff = (static_cast<size_t>(bh) * p.Lk + key) * D;
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t col0 = (part == 0 ? kColDV : kColDK) + w * (D / 2);
+                __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(part == 0 ? p.dv : p.dk) + rowoff + w * (D / 2);
+                const float mul = (part == 0) ? 1.0f : p.scale;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32(tmem_base + lane_bits + col0 + c * 32, u);
+                    tmem_wait_ld();
+                    if (valid) {
+                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            uint4 o;
+                            o.x = pack_bf16x2(__uint_as_float(u[8 * x + 0]) * mul, __uint_as_float(u[8 * x + 1]) * mul);
+                            o.y = pack_bf16x2(__uint_as_float(u[8 * x + 2]) * mul, __uint_as_float(u[8 * x + 3]) * mul);
+                            o.z = pack_bf16x2(__uint_as_float(u[8 * x + 4]) * mul, __uint_as_float(u[8 * x + 5]) * mul);
+                            o.w = pack_bf16x2(__uint_as_float(u[8 * x + 6]) * mul, __uint_as_float(u[8 * x + 7]) * mul);
+                            d4[x] = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+// ---------------------------------------------------------------- dQ
+template <int D>
+struct DqLayout {
+    using T = BwdTiles<D>;
+    static constexpr int S = T::kStages;
+    static constexpr int kQOff = 0;
+    static constexpr int kGOff = kQOff + T::kTileBytes;
+    static constexpr int kKOff = kGOff + T::kTileBytes;  // S stages
+    static constexpr int kVOff = kKOff + S * T::kTileBytes;
+    static constexpr int kBarOff = kVOff + S * T::kTileBytes;
+    // bars: qd, k[S], v[S], empty[S], s[2], dp, dsr, acc, drain
+    static constexpr int kNumBars = 1 + 3 * S + 2 + 4;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kBytes = kMiscOff + 16 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1) fa_bwd_dq(const __grid_constant__ BwdParams p) {
+    using T = BwdTiles<D>;
+    using Lay = DqLayout<D>;
+    constexpr int S = Lay::S;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem + Lay::kQOff;
+    uint8_t* sG = smem + Lay::kGOff;
+    uint8_t* sK = smem + Lay::kKOff;
+    uint8_t* sV = smem + Lay::kVOff;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
+    uint64_t* bar_qd = bars;
+    uint64_t* bar_k = bars + 1;
+    uint64_t* bar_v = bars + 1 + S;
+    uint64_t* bar_empty = bars + 1 + 2 * S;
+    uint64_t* bar_s = bars + 1 + 3 * S;  // [2]
+    uint64_t* bar_dp = bar_s + 2;
+    uint64_t* bar_dsr = bar_s + 3;
+    uint64_t* bar_acc = bar_s + 4;
+    uint64_t* bar_drain = bar_s + 5;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int BH = p.B * p.H;
+    const int nq_all = (p.Lq + 127) / 128;
+    const int qt = nq_all - 1 - static_cast<int>(blockIdx.x) / BH;  // long causal rows first
+    const int bh = static_cast<int>(blockIdx.x) % BH;
+    const int i0 = qt * 128;
+    const int off = p.Lk - p.Lq;
+    const int nk_all = (p.Lk + 127) / 128;
+    const int nk = p.causal ? min(nk_all, (min(i0 + 127, p.Lq - 1) + off) / 128 + 1) : nk_all;
+
+    // TMEM columns: S buffers [0,128) [128,256), dP [256,384), dQ [384,384+D)
+    constexpr uint32_t kColDP = 256, kColDQ = 384;
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_qd, 1);
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&bar_k[s], 1);
+            mbar_init(&bar_v[s], 1);
+            mbar_init(&bar_empty[s], 1);
+        }
+        mbar_init(&bar_s[0], 1);
+        mbar_init(&bar_s[1], 1);
+        mbar_init(bar_dp, 1);
+        mbar_init(bar_dsr, 256);
+        mbar_init(bar_acc, 1);
+        mbar_init(bar_drain, 1);
+        *abort_flag = (atomicAdd(p.status, 0) == FA_ERR_TIMEOUT) ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == 9) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 8) {
+        if (lane == 0 && !*abort_flag) {
+            tma_prefetch_desc(&p.tm_k);
+            tma_prefetch_desc(&p.tm_v);
+            mbar_arrive_expect_tx(bar_qd, 2 * T::kTileBytes);
+            for (int b = 0; b < T::kBoxes; ++b) {
+                tma_load_3d(sQ + b * T::kBoxBytes, &p.tm_q, bar_qd, b * 64, i0, bh);
+                tma_load_3d(sG + b * T::kBoxBytes, &p.tm_do, bar_qd, b * 64, i0, bh);
+            }
+            int issued = 0;
+            for (int j = 0; j < nk; ++j) {
+                const int s = j % S;
+                if (j >= S && !mbar_wait(&bar_empty[s], ((j / S) - 1) & 1, abort_flag, p.status)) break;
+                mbar_arrive_expect_tx(&bar_k[s], T::kTileBytes);
+                for (int b = 0; b < T::kBoxes; ++b)
+                    tma_load_3d(sK + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_k, &bar_k[s], b * 64, j * 128, bh);
+                mbar_arrive_expect_tx(&bar_v[s], T::kTileBytes);
+                for (int b = 0; b < T::kBoxes; ++b)
+                    tma_load_3d(sV + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_v, &bar_v[s], b * 64, j * 128, bh);
+                issued = j + 1;
+            }
+            if (*abort_flag) {
+                mbar_wait_drain(bar_qd, 0, p.status);
+                for (int j = max(0, issued - S); j < issued; ++j) {
+                    mbar_wait_drain(&bar_k[j % S], (j / S) & 1, p.status);
+                    mbar_wait_drain(&bar_v[j % S], (j / S) & 1, p.status);
+                }
+            }
+        }
+    } else if (warp == 9) {
+        if (lane == 0) {
+            constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t sQa = smem_u32(sQ), sGa = smem_u32(sG), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            auto issue_s = [&](int j) {
+                const int s = j % S;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+                    umma_ss(tmem_base + (j & 1) * 128, smem_desc_sw128(sQa + koff, 16, 1024),
+                            smem_desc_sw128(sKa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                }
+                umma_commit(&bar_s[j & 1]);
+            };
+            auto issue_dp = [&](int j) {
+                const int s = j % S;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
+                    umma_ss(tmem_base + kColDP, smem_desc_sw128(sGa + koff, 16, 1024),
+                            smem_desc_sw128(sVa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                }
+                umma_commit(bar_dp);
+            };
+            bool ok = mbar_wait(bar_qd, 0, abort_flag, p.status) && mbar_wait(&bar_k[0], 0, abort_flag, p.status);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+                ok = mbar_wait(&bar_v[0], 0, abort_flag, p.status);
+                if (ok) {
+                    tc_fence_after();
+                    issue_dp(0);
+                }
+            }
+            for (int j = 0; ok && j < nk; ++j) {
+                const int s = j % S, s1 = (j + 1) % S;
+                if (j + 1 < nk) {
+                    if (!(ok = mbar_wait(&bar_k[s1], ((j + 1) / S) & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    issue_s(j + 1);
+                }
+                // dS_j ready in S buffer j&1 (and dP_j read): dQ += dS_j K_j
+                if (!(ok = mbar_wait(bar_dsr, j & 1, abort_flag, p.status))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = tmem_base + (j & 1) * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
+                    umma_ts(tmem_base + kColDQ, a,
+                            smem_desc_sw128(sKa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                            (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bar_empty[s]);
+                if (j + 1 < nk) {
+                    if (!(ok = mbar_wait(&bar_v[s1], ((j + 1) / S) & 1, abort_flag, p.status))) break;
+                    tc_fence_after();
+                    issue_dp(j + 1);
+                }
+            }
+            if (ok) umma_commit(bar_acc);
+            umma_commit(bar_drain);
+            mbar_wait_drain(bar_drain, 0, p.status);
+        }
+    } else {
+        // ================= elementwise: thread = query row, warpgroup w = key columns [64w, 64w+64)
+        const int w = warp >> 2, wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const int row = i0 + r;
+        const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
+        const float sl2 = p.scale_log2;
+        const bool row_valid = row < p.Lq;
+        const size_t ridx = static_cast<size_t>(bh) * p.Lq + row;
+        const float lse2 = row_valid ? p.lse[ridx] * kLog2e : INFINITY;
+        const float dsum = row_valid ? p.dsum[ridx] : 0.0f;
+        const int limit = p.causal ? min(row + off, p.Lk - 1) : p.Lk - 1;  // highest permitted key
+        bool ok = true;
+        for (int j = 0; j < nk; ++j) {
+            const uint32_t tS = tmem_base + lane_bits + (j & 1) * 128 + w * 64;
+            const int k0 = j * 128 + w * 64;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[j & 1], (j >> 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            float pr[64];
+            {
+                uint32_t u[32];
+                tmem_ld32(tS, u);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) pr[x] = __uint_as_float(u[x]);
+                tmem_ld32(tS + 32, u);
+#pragma unroll
+                for (int x = 0; x < 32; ++x) pr[32 + x] = __uint_as_float(u[x]);
+                tmem_wait_ld();
+            }
+            const bool need_mask = k0 + 63 > i0 + off || k0 + 64 > p.Lk;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float v = ex2_approx(fmaf(pr[c], sl2, -lse2));
+                if (need_mask && k0 + c > limit) v = 0.0f;
+                pr[c] = v;
+            }
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, j & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                const uint32_t tDP = tmem_base + lane_bits + kColDP + w * 64;
+                uint32_t u[32], pk[32];
+                tmem_ld32(tDP, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[c] = pack_bf16x2(pr[2 * c] * (__uint_as_float(u[2 * c]) - dsum),
+                                        pr[2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum));
+                tmem_ld32(tDP + 32, u);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                    pk[16 + c] = pack_bf16x2(pr[32 + 2 * c] * (__uint_as_float(u[2 * c]) - dsum),
+                                             pr[32 + 2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum));
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(bar_dsr);
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_acc, 0, abort_flag, p.status));
+        if (ok) {
+            tc_fence_after();
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.dq) + ridx * D + w * (D / 2);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t u[32];
+                tmem_ld32(tmem_base + lane_bits + kColDQ + w * (D / 2) + c * 32, u);
+                tmem_wait_ld();
+                if (row_valid) {
+                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        uint4 o;
+                        o.x = pack_bf16x2(__uint_as_float(u[8 * x + 0]) * p.scale, __uint_as_float(u[8 * x + 1]) * p.scale);
+                        o.y = pack_bf16x2(__uint_as_float(u[8 * x + 2]) * p.scale, __uint_as_float(u[8 * x + 3]) * p.scale);
+                        o.z = pack_bf16x2(__uint_as_float(u[8 * x + 4]) * p.scale, __uint_as_float(u[8 * x + 5]) * p.scale);
+                        o.w = pack_bf16x2(__uint_as_float(u[8 * x + 6]) * p.scale, __uint_as_float(u[8 * x + 7]) * p.scale);
+                        d4[x] = o;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, 512);
+    }
+}
+
+template <int D>
+cudaError_t launch_bwd_d(const BwdParams& p, cudaStream_t stream) {
+    const long long rows = static_cast<long long>(p.B) * p.H * p.Lq;
+    const long long threads = rows * (D / 8);
+    fa_bwd_dot<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int BH = p.B * p.H;
+    const int smem1 = DkdvLayout<D>::kBytes;
+    if ((e = cudaFuncSetAttribute(fa_bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1)) !=
+        cudaSuccess)
+        return e;
+    fa_bwd_dkdv<D><<<static_cast<unsigned>(BH) * ((p.Lk + 127) / 128), kFwdThreads, smem1, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int smem2 = DqLayout<D>::kBytes;
+    if ((e = cudaFuncSetAttribute(fa_bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2)) !=
+        cudaSuccess)
+        return e;
+    fa_bwd_dq<D><<<static_cast<unsigned>(BH) * ((p.Lq + 127) / 128), kFwdThreads, smem2, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int B, int H, int Lq) {
+    const size_t n = static_cast<size_t>(B) * H * Lq * sizeof(float);
+    return (n + 255) & ~size_t(255);
+}
+
+cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream) {
+    return d == 128 ? launch_bwd_d<128>(p, stream) : launch_bwd_d<64>(p, stream);
+}
+
+}  // namespace fa

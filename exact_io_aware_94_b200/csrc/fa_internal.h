@@ -35,6 +35,28 @@ struct __align__(64) FwdParams {
     int o_dtype;
 };
 
+struct __align__(64) BwdParams {
+    CUtensorMap tm_q;   // [B*H, Lq, d] bf16, box {64, 128, 1}
+    CUtensorMap tm_k;   // [B*H, Lk, d]
+    CUtensorMap tm_v;   // [B*H, Lk, d]
+    CUtensorMap tm_do;  // [B*H, Lq, d]
+    const void* o;      // forward output, o_dtype
+    const void* dO;     // bf16 [B, H, Lq, d]
+    const float* lse;   // [B, H, Lq]
+    float* dsum;        // workspace: D_i = rowsum(dO o O), [B, H, Lq]
+    void* dq;           // bf16 outputs
+    void* dk;
+    void* dv;
+    int* status;
+    int B, H, Lq, Lk;
+    float scale, scale_log2;
+    int causal;
+    int o_dtype;
+};
+
+size_t bwd_workspace_bytes(int B, int H, int Lq);
+cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream);
+
 // Decode: keys of each sequence are cut into chunks of kDecodeSplit keys.
 constexpr int kDecodeSplit = 1024;
 constexpr int kDecodeThreads = 256;
