@@ -35,6 +35,8 @@ FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
 FA_ERR_DEVICE = 6
 FA_ERR_KV_LEN = 7
+FA_ERR_TOO_LARGE = 8
+FA_NOALLOC_MAX_ROWS = 1 << 20
 FA_DT_BF16 = 0
 FA_DT_F32 = 1
 
@@ -65,6 +67,8 @@ def load_library():
     lib.fa_backward_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_backward.restype = i
     lib.fa_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, sz, vp]
+    lib.fa_backward_noalloc.restype = i
+    lib.fa_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
     lib.fa_decode_workspace_size.restype = sz
     lib.fa_decode_workspace_size.argtypes = [i, i, i, i]
     lib.fa_decode.restype = i
@@ -113,6 +117,13 @@ def fa_backward(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal,
     return load_library().fa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
                                       _ptr(dk), _ptr(dv), B, H, Lq, Lk, d, float(scale), int(causal),
                                       int(o_dtype), _ptr(workspace), int(workspace_bytes), _stream(stream))
+
+
+def fa_backward_noalloc(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, o_dtype,
+                        stream=None) -> int:
+    return load_library().fa_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dO), _ptr(lse), _ptr(dq),
+                                              _ptr(dk), _ptr(dv), B, H, Lq, Lk, d, float(scale), int(causal),
+                                              int(o_dtype), _stream(stream))
 
 
 def fa_decode_workspace_size(B, H, cap, d) -> int:

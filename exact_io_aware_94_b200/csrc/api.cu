@@ -88,6 +88,19 @@ bool dims_ok(int B, int H, int L, int d) {
 }
 
 }  // namespace
+
+// Internal helpers shared with other translation units of this library.
+int prepare_device(int** status_ptr) {
+    DeviceState* st = nullptr;
+    const int rc = device_state(&st);
+    if (rc == FA_OK) *status_ptr = st->status_ptr;
+    return rc;
+}
+int encode_tile_map(CUtensorMap* map, const void* base, int BH, int L, int d, int box_rows) {
+    return encode_rows_map(map, base, BH, L, d, box_rows);
+}
+bool shape_ok(int B, int H, int L, int d) { return dims_ok(B, H, L, d); }
+
 }  // namespace fa
 
 using namespace fa;
@@ -104,6 +117,8 @@ const char* fa_status_string(int status) {
         case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded wait inside a kernel ran out";
         case FA_ERR_DEVICE: return "FA_ERR_DEVICE: current device is not compute capability 10.0 (sm_100a)";
         case FA_ERR_KV_LEN: return "FA_ERR_KV_LEN: a decode cache length was outside [0, cap]";
+        case FA_ERR_TOO_LARGE:
+            return "FA_ERR_TOO_LARGE: B*H*Lq exceeds FA_NOALLOC_MAX_ROWS, the fixed scratch of fa_backward_noalloc";
         default: return "unknown fa_status";
     }
 }

@@ -55,6 +55,11 @@ struct __align__(64) BwdParams {
 };
 
 size_t bwd_workspace_bytes(int B, int H, int Lq);
+
+// Helpers implemented in api.cu for the other entry points.
+int prepare_device(int** status_ptr);
+int encode_tile_map(CUtensorMap* map, const void* base, int BH, int L, int d, int box_rows);
+bool shape_ok(int B, int H, int L, int d);
 cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream);
 
 // Decode: keys of each sequence are cut into chunks of kDecodeSplit keys.

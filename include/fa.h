@@ -57,7 +57,8 @@ typedef enum {
     FA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
     FA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
     FA_ERR_DEVICE = 6,      /* current device is not compute capability 10.0 */
-    FA_ERR_KV_LEN = 7       /* device: a decode cache length was outside [0, cap] (clamped) */
+    FA_ERR_KV_LEN = 7,      /* device: a decode cache length was outside [0, cap] (clamped) */
+    FA_ERR_TOO_LARGE = 8    /* problem larger than the fixed scratch of fa_backward_noalloc */
 } fa_status;
 
 enum { FA_DT_BF16 = 0, FA_DT_F32 = 1 };
@@ -92,6 +93,32 @@ size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d);
 int fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                 void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
                 int o_dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_backward without a workspace argument, for callers that cannot allocate
+ * device memory at all: for example a plugin whose host framework owns every
+ * device allocation and offers no workspace hook, or a latency-critical loop in
+ * which cudaMalloc's implicit device synchronisation is not acceptable.  The
+ * pages have no counterpart to this call; it is a packaging variant of
+ * fa_backward.
+ *
+ * Same arguments, layout and results as fa_backward.  Its scratch (the per-row
+ * statistic D, 4 bytes per query row) lives in a statically allocated device
+ * array of FA_NOALLOC_MAX_ROWS floats (4 MiB) that every GPU loading this
+ * library holds until the process exits.  No call allocates or frees memory.
+ *   - B*H*Lq > FA_NOALLOC_MAX_ROWS returns FA_ERR_TOO_LARGE; nothing is launched.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once; make that first call before any stream
+ *     capture.
+ *   - Every call on a device shares the one array, and the array keeps the last
+ *     call's contents.  Each call writes every D_i it reads before reading it,
+ *     so nothing has to start at zero.  Calls whose kernels overlap on the GPU
+ *     (for example on two streams at once) race on the array: serialise them.
+ */
+#define FA_NOALLOC_MAX_ROWS (1 << 20)
+int fa_backward_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                        const float* lse, void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d,
+                        float scale, int causal, int o_dtype, void* stream);
 
 /*
  * Workspace bytes fa_decode needs: split-KV partial results (fp32 output
