@@ -156,7 +156,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
-    cudaError_t e = launch_fwd(p, d, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_fwd(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -88,7 +88,7 @@ struct DkdvLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1) fa_bwd_dkdv(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_constant__ BwdParams p) {
     using T = BwdTiles<D>;
     using Lay = DkdvLayout<D>;
     constexpr int S = Lay::S;
@@ -372,7 +372,7 @@ struct DqLayout {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kFwdThreads, 1) fa_bwd_dq(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constant__ BwdParams p) {
     using T = BwdTiles<D>;
     using Lay = DqLayout<D>;
     constexpr int S = Lay::S;
@@ -631,13 +631,13 @@ cudaError_t launch_bwd_d(const BwdParams& p, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(fa_bwd_dkdv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1)) !=
         cudaSuccess)
         return e;
-    fa_bwd_dkdv<D><<<static_cast<unsigned>(BH) * ((p.Lk + 127) / 128), kFwdThreads, smem1, stream>>>(p);
+    fa_bwd_dkdv<D><<<static_cast<unsigned>(BH) * ((p.Lk + 127) / 128), kBwdThreads, smem1, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int smem2 = DqLayout<D>::kBytes;
     if ((e = cudaFuncSetAttribute(fa_bwd_dq<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2)) !=
         cudaSuccess)
         return e;
-    fa_bwd_dq<D><<<static_cast<unsigned>(BH) * ((p.Lq + 127) / 128), kFwdThreads, smem2, stream>>>(p);
+    fa_bwd_dq<D><<<static_cast<unsigned>(BH) * ((p.Lq + 127) / 128), kBwdThreads, smem2, stream>>>(p);
     return cudaGetLastError();
 }
 

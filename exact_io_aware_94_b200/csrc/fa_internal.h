@@ -19,7 +19,14 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr int kFwdBM = 128;
 constexpr int kFwdBN = 128;
 constexpr int kFwdRowsPerCta = 2 * kFwdBM;
-constexpr int kFwdThreads = 320;  // 2 softmax warpgroups + TMA warp + MMA warp
+constexpr int kFwdThreads = 384;  // 2 softmax warpgroups + a warpgroup holding the TMA and MMA warps
+constexpr int kBwdThreads = 320;  // 2 elementwise warpgroups + TMA warp + MMA warp
+// Register split of the forward kernel (setmaxnreg): the two softmax warpgroups
+// grow to kFwdRegsSoftmax, the TMA/MMA warpgroup shrinks to kFwdRegsOther.  The
+// launch allocation must cover the split: kFwdThreads x (registers the kernel is
+// compiled with) >= 2*128*kFwdRegsSoftmax + 128*kFwdRegsOther; launch_fwd checks.
+constexpr int kFwdRegsSoftmax = 216;
+constexpr int kFwdRegsOther = 72;
 
 struct __align__(64) FwdParams {
     CUtensorMap tm_q;  // [B*H, Lq, d] bf16, box {64, 128, 1}, 128B swizzle
@@ -89,6 +96,6 @@ void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, in
 cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 
 int fwd_smem_bytes(int d);
-cudaError_t launch_fwd(const FwdParams& p, int d, cudaStream_t stream);
+cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
 
 }  // namespace fa

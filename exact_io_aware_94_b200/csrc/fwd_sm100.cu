@@ -6,23 +6,31 @@
 // update the running max m and running sum l per row, rescale the unnormalised
 // output O~ when the max moves, accumulate P~ V, and divide by l at the end.
 //
-// B200 mapping (one CTA = 256 query rows of one (b, h)):
-//   warp 8      TMA producer: Q tiles once, then K_j / V_j into a smem ring.
+// B200 mapping.  A work unit is 256 query rows of one (b, h): two 128-row Q
+// tiles, one per softmax warpgroup.  The kernel is persistent (one CTA per SM)
+// and walks a static, balanced share of the units; the next unit's Q is loaded as soon as
+// the current unit's last S MMA has been issued, so loads, MMAs and the
+// epilogue of consecutive units overlap.
+//   warp 8      TMA producer: Q tiles per unit, K_j / V_j through a smem ring.
 //   warp 9      MMA issuer (one thread): S_w = Q_w K_j^T into TMEM (SS MMA),
 //               O_w += P_w V_j with P_w read from TMEM (TS MMA).
-//   warps 0-3   softmax warpgroup 0 (rows 0..127 of the CTA), warps 4-7
+//   warps 10-11 idle (they complete the third warpgroup, whose registers
+//               setmaxnreg hands to the softmax warpgroups).
+//   warps 0-3   softmax warpgroup 0 (rows 0..127 of the unit), warps 4-7
 //               warpgroup 1 (rows 128..255).  One thread owns one row: it loads
 //               its score row from TMEM, applies the mask, updates m and l,
-//               rescales its O~ row in TMEM when needed, and writes bf16 P~
-//               back over its score row for the PV MMA.
+//               rescales its O~ row in TMEM when needed, writes bf16 P~ back
+//               over its score row for the PV MMA, and finally stores O, LSE.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+d) O1 [256+d,256+2d).
 //
 // Rescaling is deferred while the running max has grown by no more than
 // 2^kRescaleLog2 in exp2 units: O = O~ / l holds for any common reference
 // value, so the result is unchanged; only overflow headroom is spent.
-// O is normalised by the sum of the bf16-rounded P~ that the MMA consumes, so
-// numerator and denominator use the same weights; the LSE uses the sum of the
-// unrounded P~.
+// The LSE uses the running sum of the unrounded P~.  O is normalised by that
+// sum plus, per tile, the bf16 rounding error of the tile's largest P~ (the
+// term that dominates a peaky row), so numerator and denominator weigh the
+// dominant key alike.  Optionally some exponentials run as a polynomial on the
+// FMA pipe instead of MUFU (off by default, see kEmuPer8).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,6 +43,16 @@ namespace {
 
 constexpr float kRescaleLog2 = 8.0f;
 
+// Of every 8 consecutive score columns, the last kEmuPer8 take their
+// exponential on the FMA pipe (polynomial) instead of MUFU.  Measured on B200
+// the softmax is issue-bound rather than MUFU-bound (every fraction tried
+// from 1/8 to 3/8 was slower), so the default is 0.
+#ifndef FA_FWD_EMU_PER8
+#define FA_FWD_EMU_PER8 0
+#endif
+constexpr int kEmuPer8 = FA_FWD_EMU_PER8;
+__device__ __forceinline__ constexpr bool emulated_col(int c) { return (c & 7) >= 8 - kEmuPer8; }
+
 template <int D>
 struct FwdLayout {
     static constexpr int kBoxBytes = 128 * 64 * 2;     // one TMA box: 128 rows x 64 bf16
@@ -45,11 +63,45 @@ struct FwdLayout {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    // barriers: q, k[S], v[S], empty[S], s[2], p[2], o[2], drain
-    static constexpr int kNumBars = 1 + 3 * kStages + 2 + 2 + 2 + 1;
+    // barriers: q, q_free, k[S], v[S], empty[S], s[2], p[2], o[2], o_free[2], drain
+    static constexpr int kNumBars = 2 + 3 * kStages + 2 * 4 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16 + 1024;  // + tmem slot/abort + alignment slack
 };
+
+// One work unit: which (b*H + h), which pair of 128-row tiles, how many KV tiles each needs.
+struct Unit {
+    int bh, i0, n_kv0, n_kv1;
+};
+
+// Units in a fixed global order: longest causal rows first (pair index
+// descending), heads interleaved.
+__device__ __forceinline__ Unit unit_of(const FwdParams& p, int u) {
+    const int BH = p.B * p.H;
+    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    Unit r;
+    const int pair = n_pairs - 1 - u / BH;
+    r.bh = u % BH;
+    r.i0 = pair * kFwdRowsPerCta;
+    const int n_kv_all = (p.Lk + kFwdBN - 1) / kFwdBN;
+    const int off = p.Lk - p.Lq;  // causal: query i sits at key position i + off
+    int n[2];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const int first = r.i0 + w * kFwdBM;
+        if (first >= p.Lq) {
+            n[w] = 0;
+        } else if (p.causal) {
+            const int last = min(first + kFwdBM - 1, p.Lq - 1);
+            n[w] = min(n_kv_all, (last + off) / kFwdBN + 1);
+        } else {
+            n[w] = n_kv_all;
+        }
+    }
+    r.n_kv0 = n[0];
+    r.n_kv1 = n[1];
+    return r;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -62,45 +114,34 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint8_t* sV = smem + Lay::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
     uint64_t* bar_q = bars;
-    uint64_t* bar_k = bars + 1;
-    uint64_t* bar_v = bars + 1 + S;
-    uint64_t* bar_empty = bars + 1 + 2 * S;
-    uint64_t* bar_s = bars + 1 + 3 * S;
+    uint64_t* bar_q_free = bars + 1;
+    uint64_t* bar_k = bars + 2;
+    uint64_t* bar_v = bars + 2 + S;
+    uint64_t* bar_empty = bars + 2 + 2 * S;
+    uint64_t* bar_s = bars + 2 + 3 * S;
     uint64_t* bar_p = bar_s + 2;
     uint64_t* bar_o = bar_p + 2;
-    uint64_t* bar_drain = bar_o + 2;
+    uint64_t* bar_ofree = bar_o + 2;
+    uint64_t* bar_drain = bar_ofree + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work unit: (b*H + h, pair of 128-row Q tiles), longest causal rows first
-    const int BH = p.B * p.H;
-    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
-    const int pair = n_pairs - 1 - static_cast<int>(blockIdx.x) / BH;
-    const int bh = static_cast<int>(blockIdx.x) % BH;
-    const int i0 = pair * kFwdRowsPerCta;
-    const int n_kv_all = (p.Lk + kFwdBN - 1) / kFwdBN;
-    const int off = p.Lk - p.Lq;  // causal: query i sits at key position i + off
-    int n_kv[2];
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-        const int first = i0 + w * kFwdBM;
-        if (first >= p.Lq) {
-            n_kv[w] = 0;
-        } else if (p.causal) {
-            const int last = min(first + kFwdBM - 1, p.Lq - 1);
-            n_kv[w] = min(n_kv_all, (last + off) / kFwdBN + 1);
-        } else {
-            n_kv[w] = n_kv_all;
-        }
-    }
-    const int n_max = max(n_kv[0], n_kv[1]);
+    const int n_units = p.B * p.H * ((p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+    // Static boustrophedon assignment: in round r this CTA takes unit
+    // r*G + c (r even) or r*G + G-1-c (r odd).  Over the heavy-first order this
+    // balances the causal work across CTAs without any shared counter.
+    auto snake_unit = [&](int r) {
+        const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+        return r * g + ((r & 1) ? g - 1 - c : c);
+    };
+    const int off = p.Lk - p.Lq;
 
     // ---- setup
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
+        mbar_init(bar_q_free, 1);
         for (int s = 0; s < S; ++s) {
             mbar_init(&bar_k[s], 1);
             mbar_init(&bar_v[s], 1);
@@ -110,6 +151,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             mbar_init(&bar_s[w], 1);
             mbar_init(&bar_p[w], 4 * 32);
             mbar_init(&bar_o[w], 1);
+            mbar_init(&bar_ofree[w], 4 * 32);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = (atomicAdd(p.status, 0) == FA_ERR_TIMEOUT) ? 1 : 0;
@@ -129,49 +171,56 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
+    // Registers move from the TMA/MMA warpgroup (warps 8-11) to the softmax
+    // warpgroups (warps 0-7); each setmaxnreg sits in its own role's branch.
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kFwdRegsOther));
+    }
     if (warp == 8) {
         // ================= TMA producer =================
         if (lane == 0 && !*abort_flag) {
-            uint32_t q_bytes = 0;
-#pragma unroll
-            for (int w = 0; w < 2; ++w)
-                if (n_kv[w] > 0) q_bytes += Lay::kTileBytes;
-            if (q_bytes) {
+            int kc = 0;       // K/V tiles issued so far (ring position)
+            int q_iter = 0;   // units whose Q has been requested
+            bool ok = true;
+            for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+                const Unit un = unit_of(p, u);
+                const int n_max = max(un.n_kv0, un.n_kv1);
+                // the previous unit's S MMAs must be done with the Q buffer
+                if (q_iter > 0 && !(ok = mbar_wait(bar_q_free, (q_iter - 1) & 1, abort_flag, p.status))) break;
+                const uint32_t q_bytes = (un.n_kv1 > 0 ? 2 : 1) * Lay::kTileBytes;
                 mbar_arrive_expect_tx(bar_q, q_bytes);
-#pragma unroll
                 for (int w = 0; w < 2; ++w) {
-                    if (n_kv[w] == 0) continue;
+                    if ((w == 0 ? un.n_kv0 : un.n_kv1) == 0) continue;
                     for (int b = 0; b < Lay::kBoxes; ++b)
                         tma_load_3d(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, bar_q, b * 64,
-                                    i0 + w * kFwdBM, bh);
+                                    un.i0 + w * kFwdBM, un.bh);
                 }
-            }
-            int issued = 0;
-            for (int j = 0; j < n_max; ++j) {
-                const int s = j % S;
-                if (j >= S && !mbar_wait(&bar_empty[s], ((j / S) - 1) & 1, abort_flag, p.status)) break;
-                mbar_arrive_expect_tx(&bar_k[s], Lay::kTileBytes);
-                for (int b = 0; b < Lay::kBoxes; ++b)
-                    tma_load_3d(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
-                                j * kFwdBN, bh);
-                mbar_arrive_expect_tx(&bar_v[s], Lay::kTileBytes);
-                for (int b = 0; b < Lay::kBoxes; ++b)
-                    tma_load_3d(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
-                                j * kFwdBN, bh);
-                issued = j + 1;
+                ++q_iter;
+                for (int j = 0; j < n_max; ++j, ++kc) {
+                    const int s = kc % S;
+                    if (kc >= S && !(ok = mbar_wait(&bar_empty[s], ((kc / S) - 1) & 1, abort_flag, p.status))) break;
+                    mbar_arrive_expect_tx(&bar_k[s], Lay::kTileBytes);
+                    for (int b = 0; b < Lay::kBoxes; ++b)
+                        tma_load_3d(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
+                                    j * kFwdBN, un.bh);
+                    mbar_arrive_expect_tx(&bar_v[s], Lay::kTileBytes);
+                    for (int b = 0; b < Lay::kBoxes; ++b)
+                        tma_load_3d(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
+                                    j * kFwdBN, un.bh);
+                }
             }
             if (*abort_flag) {
                 // Let copies already in flight land before the CTA's smem goes away.
-                if (q_bytes) mbar_wait_drain(bar_q, 0, p.status);
-                for (int j = max(0, issued - S); j < issued; ++j) {
-                    mbar_wait_drain(&bar_k[j % S], (j / S) & 1, p.status);
-                    mbar_wait_drain(&bar_v[j % S], (j / S) & 1, p.status);
+                if (q_iter > 0) mbar_wait_drain(bar_q, (q_iter - 1) & 1, p.status);
+                for (int t = max(0, kc - S); t < kc; ++t) {
+                    mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
+                    mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
                 }
             }
         }
     } else if (warp == 9) {
         // ================= MMA issuer =================
-        if (lane == 0 && n_max > 0) {
+        if (lane == 0) {
             constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
@@ -196,173 +245,228 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     umma_ts(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = mbar_wait(bar_q, 0, abort_flag, p.status) && mbar_wait(&bar_k[0], 0, abort_flag, p.status);
-            if (ok) {
+            int kc = 0;               // K/V ring position
+            int q_iter = 0;           // units started
+            int tp[2] = {0, 0};       // P tiles consumed per warpgroup
+            int units_w[2] = {0, 0};  // units whose O_w was handed to the epilogue
+            bool ok = true;
+            for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+                const Unit un = unit_of(p, u);
+                const int n0 = un.n_kv0, n1 = un.n_kv1;
+                const int n_max = max(n0, n1);
+                if (!(ok = mbar_wait(bar_q, q_iter & 1, abort_flag, p.status))) break;
+                ++q_iter;
+                if (!(ok = mbar_wait(&bar_k[kc % S], (kc / S) & 1, abort_flag, p.status))) break;
                 tc_fence_after();
+                issue_s(0, kc % S);
+                if (n1 > 0) issue_s(1, kc % S);
+                if (n_max == 1) umma_commit(bar_q_free);
+                for (int j = 0; ok && j < n_max; ++j) {
+                    const int s = (kc + j) % S;
+                    const int s1 = (kc + j + 1) % S;
+                    if (!(ok = mbar_wait(&bar_v[s], ((kc + j) / S) & 1, abort_flag, p.status))) break;
+                    bool k_ready = false;
 #pragma unroll
-                for (int w = 0; w < 2; ++w)
-                    if (n_kv[w] > 0) issue_s(w, 0);
-            }
-            for (int j = 0; ok && j < n_max; ++j) {
-                const int s = j % S;
-                const int s1 = (j + 1) % S;
-                if (!mbar_wait(&bar_v[s], (j / S) & 1, abort_flag, p.status)) break;
-                const bool more = (j + 1 < n_max);
-                bool k_ready = false;
-#pragma unroll
-                for (int w = 0; w < 2; ++w) {
-                    if (j < n_kv[w]) {
-                        if (!(ok = mbar_wait(&bar_p[w], j & 1, abort_flag, p.status))) break;
-                        tc_fence_after();
-                        issue_pv(w, s, j);
-                        if (j == n_kv[w] - 1) umma_commit(&bar_o[w]);
-                    }
-                    if (j + 1 < n_kv[w]) {
-                        if (!k_ready) {
-                            if (!(ok = mbar_wait(&bar_k[s1], ((j + 1) / S) & 1, abort_flag, p.status))) break;
+                    for (int w = 0; w < 2; ++w) {
+                        const int nw = (w == 0) ? n0 : n1;
+                        if (j < nw) {
+                            if (j == 0 && units_w[w] > 0) {
+                                // O_w still holds the previous unit until its epilogue has read it
+                                if (!(ok = mbar_wait(&bar_ofree[w], (units_w[w] - 1) & 1, abort_flag, p.status)))
+                                    break;
+                            }
+                            if (!(ok = mbar_wait(&bar_p[w], tp[w] & 1, abort_flag, p.status))) break;
+                            ++tp[w];
                             tc_fence_after();
-                            k_ready = true;
+                            issue_pv(w, s, j);
+                            if (j == nw - 1) {
+                                umma_commit(&bar_o[w]);
+                                ++units_w[w];
+                            }
                         }
-                        issue_s(w, s1);
+                        if (j + 1 < nw) {
+                            if (!k_ready) {
+                                if (!(ok = mbar_wait(&bar_k[s1], ((kc + j + 1) / S) & 1, abort_flag, p.status)))
+                                    break;
+                                tc_fence_after();
+                                k_ready = true;
+                            }
+                            issue_s(w, s1);
+                        }
                     }
+                    if (!ok) break;
+                    if (j + 2 == n_max) umma_commit(bar_q_free);  // last S of this unit issued
+                    umma_commit(&bar_empty[s]);
                 }
-                (void)more;
-                umma_commit(&bar_empty[s]);
+                kc += n_max;
             }
             // Drain: every MMA issued by this thread completes before TMEM is freed.
             umma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.status);
         }
-    } else {
+    } else if (warp < 8) {
         // ================= softmax warpgroups =================
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kFwdRegsSoftmax));
         const int w = warp >> 2;
         const int wq = warp & 3;
         const int row_in_tile = wq * 32 + lane;
-        const int row = i0 + w * kFwdBM + row_in_tile;
         const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t t_s = tmem_base + lane_bits + w * 128;
         const uint32_t t_o = tmem_base + lane_bits + 256 + w * D;
         const float sl2 = p.scale_log2;
-        const int tile_first_row = i0 + w * kFwdBM;
-        const int n = (w == 0) ? n_kv[0] : n_kv[1];
-
-        float m_ref = -INFINITY;  // running max of raw scores q.k (reference for P~)
-        float l = 0.0f;           // running sum of P~ as rounded to bf16: normalises O
-        float l_exact = 0.0f;     // running sum of P~ before rounding: gives the LSE
+        int ts = 0;      // S tiles consumed by this warpgroup
+        int nunits = 0;  // units finished by this warpgroup
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            // warp-uniform outcome: the TMEM accesses below are warp-collective
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[w], j & 1, abort_flag, p.status));
-            if (!ok) break;
-            tc_fence_after();
-            float s[kFwdBN];
-            {
-                uint32_t r[32];
+        for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+            const Unit un = unit_of(p, u);
+            const int n = (w == 0) ? un.n_kv0 : un.n_kv1;
+            if (n == 0) continue;
+            const int tile_first_row = un.i0 + w * kFwdBM;
+            const int row = tile_first_row + row_in_tile;
+            const int limit = p.causal ? min(row + off, p.Lk - 1) : p.Lk - 1;  // highest permitted key
+
+            float m_ref = -INFINITY;  // running max of raw scores q.k (reference for P~)
+            float l = 0.0f;           // running sum of the unrounded P~: gives the LSE
+            float corr = 0.0f;        // sum over tiles of (bf16(P~_max) - P~_max): l + corr normalises O
+            for (int j = 0; j < n; ++j, ++ts) {
+                // warp-uniform outcome: the TMEM accesses below are warp-collective
+                ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[w], ts & 1, abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                float s[kFwdBN];
+                {
+                    uint32_t r[32];
 #pragma unroll
-                for (int c = 0; c < kFwdBN / 32; ++c) {
-                    tmem_ld32(t_s + c * 32, r);
+                    for (int c = 0; c < kFwdBN / 32; ++c) {
+                        tmem_ld32(t_s + c * 32, r);
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
+                        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(r[x]);
+                    }
+                    tmem_wait_ld();
                 }
-                tmem_wait_ld();
-            }
-            const int kv0 = j * kFwdBN;
-            const bool need_mask =
-                (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) || (kv0 + kFwdBN > p.Lk);
-            if (need_mask) {
-                const int limit = p.causal ? min(row + off, p.Lk - 1) : p.Lk - 1;
+                const int kv0 = j * kFwdBN;
+                const bool need_mask =
+                    (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) || (kv0 + kFwdBN > p.Lk);
+                if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < kFwdBN; ++c)
-                    if (kv0 + c > limit) s[c] = -INFINITY;
-            }
-            float mx;
-            {
-                float mp[8];
+                    for (int c = 0; c < kFwdBN; ++c)
+                        if (kv0 + c > limit) s[c] = -INFINITY;
+                }
+                // Row max, kept separately over the columns whose exponential runs
+                // on MUFU (mx_a) and on the FMA pipe (mx_b), so the rounding
+                // correction below can redo the max element on the same path.
+                float mx_a, mx_b;
+                {
+                    float ma[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                    float mb2[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                for (int x = 0; x < 8; ++x) mp[x] = s[x];
-#pragma unroll
-                for (int c = 8; c < kFwdBN; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-                mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                           fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            }
-            const float m_new = fmaxf(m_ref, mx);
-            const bool want = (m_ref == -INFINITY) ? (m_new != -INFINITY) : ((m_new - m_ref) * sl2 > kRescaleLog2);
-            if (__any_sync(0xffffffffu, want)) {
-                const float alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
-                l *= alpha;
-                l_exact *= alpha;
-                m_ref = m_new;
-                if (j > 0) {
-                    // Small chunks: the score row stays live in registers meanwhile.
+                    for (int c = 0; c < kFwdBN; c += 2) {
+                        if (emulated_col(c)) {
+                            mb2[(c >> 3) & 1] = fmax3(mb2[(c >> 3) & 1], s[c], s[c + 1]);
+                        } else {
+                            ma[(c >> 1) & 3] = fmax3(ma[(c >> 1) & 3], s[c], s[c + 1]);
+                        }
+                    }
+                    mx_a = fmax3(ma[0], ma[1], fmaxf(ma[2], ma[3]));
+                    mx_b = fmaxf(mb2[0], mb2[1]);
+                }
+                const float mx = fmaxf(mx_a, mx_b);
+                const float m_new = fmaxf(m_ref, mx);
+                const bool want =
+                    (m_ref == -INFINITY) ? (m_new != -INFINITY) : ((m_new - m_ref) * sl2 > kRescaleLog2);
+                if (__any_sync(0xffffffffu, want)) {
+                    const float alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
+                    l *= alpha;
+                    corr *= alpha;
+                    m_ref = m_new;
+                    if (j > 0) {
+                        // Small chunks: the score row stays live in registers meanwhile.
 #pragma unroll 1
-                    for (int c = 0; c < D / 8; ++c) {
-                        uint32_t r[8];
-                        tmem_ld8(t_o + c * 8, r);
-                        tmem_wait_ld();
+                        for (int c = 0; c < D / 8; ++c) {
+                            uint32_t r[8];
+                            tmem_ld8(t_o + c * 8, r);
+                            tmem_wait_ld();
 #pragma unroll
-                        for (int x = 0; x < 8; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-                        tmem_st8(t_o + c * 8, r);
+                            for (int x = 0; x < 8; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
+                            tmem_st8(t_o + c * 8, r);
+                        }
                     }
                 }
-            }
-            const float mb = (m_ref == -INFINITY) ? 0.0f : m_ref * sl2;
-            uint32_t pk[kFwdBN / 2];
-            float lp[4] = {0.f, 0.f, 0.f, 0.f};  // sums of the bf16-rounded P~ (what the MMA sees)
-            float le[4] = {0.f, 0.f, 0.f, 0.f};  // sums of the unrounded P~ (for the LSE)
+                const float mb = (m_ref == -INFINITY) ? 0.0f : m_ref * sl2;
+                uint32_t pk[kFwdBN / 2];
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int c = 0; c < kFwdBN / 2; ++c) {
-                const float p0 = ex2_approx(fmaf(s[2 * c], sl2, -mb));
-                const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, -mb));
-                pk[c] = pack_bf16x2(p0, p1);
-                lp[c & 3] += bf16lo_to_f32(pk[c]) + bf16hi_to_f32(pk[c]);
-                le[c & 3] += p0 + p1;
+                for (int c = 0; c < kFwdBN; c += 2) {
+                    const float x0 = fmaf(s[c], sl2, -mb);
+                    const float x1 = fmaf(s[c + 1], sl2, -mb);
+                    float p0 = emulated_col(c) ? exp2_poly(x0) : ex2_approx(x0);
+                    float p1 = emulated_col(c + 1) ? exp2_poly(x1) : ex2_approx(x1);
+                    if (need_mask) {  // exact zeros for masked keys
+                        p0 = (kv0 + c > limit) ? 0.0f : p0;
+                        p1 = (kv0 + c + 1 > limit) ? 0.0f : p1;
+                    }
+                    ls[(c >> 1) & 3] += p0 + p1;
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                }
+                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                {
+                    // The tile's largest P~ dominates its row's rounding error: account
+                    // for its bf16 rounding in the normaliser of O (recomputed on the
+                    // same exponential path as the element itself).
+                    const float xm = fmaf(mx, sl2, -mb);
+                    const float pmax = (mx == -INFINITY) ? 0.0f : (mx_b > mx_a ? exp2_poly(xm) : ex2_approx(xm));
+                    corr += round_bf16(pmax) - pmax;
+                }
+                tmem_st16(t_s + 0, pk + 0);
+                tmem_st16(t_s + 16, pk + 16);
+                tmem_st16(t_s + 32, pk + 32);
+                tmem_st16(t_s + 48, pk + 48);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bar_p[w]);
             }
-            l += (lp[0] + lp[1]) + (lp[2] + lp[3]);
-            l_exact += (le[0] + le[1]) + (le[2] + le[3]);
-            tmem_st16(t_s + 0, pk + 0);
-            tmem_st16(t_s + 16, pk + 16);
-            tmem_st16(t_s + 32, pk + 32);
-            tmem_st16(t_s + 48, pk + 48);
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&bar_p[w]);
-        }
+            if (!ok) break;
 
-        // ---- epilogue: O = O~ / l, LSE = scale * m + ln l
-        if (n > 0 && ok) ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[w], 0, abort_flag, p.status));
-        if (n > 0 && ok) {
+            // ---- epilogue: O = O~ / l, LSE = scale * m + ln l
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_o[w], nunits & 1, abort_flag, p.status));
+            if (!ok) break;
+            ++nunits;
             tc_fence_after();
-            const bool valid = row < p.Lq;
-            const float inv_l = 1.0f / l;
-            const size_t row_idx = static_cast<size_t>(bh) * p.Lq + row;
+            uint32_t ov[D];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(t_o + c * 32, r);
-                tmem_wait_ld();
-                if (valid) {
-                    if (p.o_dtype == FA_DT_F32) {
-                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row_idx * D + c * 32);
 #pragma unroll
-                        for (int x = 0; x < 8; ++x)
-                            dst[x] = make_float4(__uint_as_float(r[4 * x]) * inv_l, __uint_as_float(r[4 * x + 1]) * inv_l,
-                                                 __uint_as_float(r[4 * x + 2]) * inv_l,
-                                                 __uint_as_float(r[4 * x + 3]) * inv_l);
-                    } else {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D + c * 32);
+                for (int x = 0; x < 32; ++x) ov[c * 32 + x] = r[x];
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bar_ofree[w]);  // O_w may now be overwritten by the next unit's PV
+            if (row < p.Lq) {
+                const float inv_l = 1.0f / (l + corr);
+                const size_t row_idx = static_cast<size_t>(un.bh) * p.Lq + row;
+                if (p.o_dtype == FA_DT_F32) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row_idx * D);
 #pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            uint4 u;
-                            u.x = pack_bf16x2(__uint_as_float(r[8 * x + 0]) * inv_l, __uint_as_float(r[8 * x + 1]) * inv_l);
-                            u.y = pack_bf16x2(__uint_as_float(r[8 * x + 2]) * inv_l, __uint_as_float(r[8 * x + 3]) * inv_l);
-                            u.z = pack_bf16x2(__uint_as_float(r[8 * x + 4]) * inv_l, __uint_as_float(r[8 * x + 5]) * inv_l);
-                            u.w = pack_bf16x2(__uint_as_float(r[8 * x + 6]) * inv_l, __uint_as_float(r[8 * x + 7]) * inv_l);
-                            dst[x] = u;
-                        }
+                    for (int x = 0; x < D / 4; ++x)
+                        dst[x] = make_float4(__uint_as_float(ov[4 * x]) * inv_l, __uint_as_float(ov[4 * x + 1]) * inv_l,
+                                             __uint_as_float(ov[4 * x + 2]) * inv_l,
+                                             __uint_as_float(ov[4 * x + 3]) * inv_l);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D);
+#pragma unroll
+                    for (int x = 0; x < D / 8; ++x) {
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(ov[8 * x + 0]) * inv_l, __uint_as_float(ov[8 * x + 1]) * inv_l);
+                        v4.y = pack_bf16x2(__uint_as_float(ov[8 * x + 2]) * inv_l, __uint_as_float(ov[8 * x + 3]) * inv_l);
+                        v4.z = pack_bf16x2(__uint_as_float(ov[8 * x + 4]) * inv_l, __uint_as_float(ov[8 * x + 5]) * inv_l);
+                        v4.w = pack_bf16x2(__uint_as_float(ov[8 * x + 6]) * inv_l, __uint_as_float(ov[8 * x + 7]) * inv_l);
+                        dst[x] = v4;
                     }
                 }
+                p.lse[row_idx] = m_ref * p.scale + logf(l);
             }
-            if (valid) p.lse[row_idx] = m_ref * p.scale + logf(l_exact);
         }
     }
 
@@ -374,22 +478,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
 }
 
+// The setmaxnreg split only works if the block was launched with at least as
+// many registers as the split hands out; otherwise the increase would wait
+// forever.  Refuse to launch a build whose register count does not cover it.
+template <typename K>
+cudaError_t check_register_split(K kernel) {
+    cudaFuncAttributes a{};
+    cudaError_t e = cudaFuncGetAttributes(&a, kernel);
+    if (e != cudaSuccess) return e;
+    const long long pool = static_cast<long long>(a.numRegs) * kFwdThreads;
+    const long long need = 2LL * 128 * kFwdRegsSoftmax + 128LL * kFwdRegsOther;
+    return pool >= need ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 }  // namespace
 
 int fwd_smem_bytes(int d) { return d == 128 ? FwdLayout<128>::kBytes : FwdLayout<64>::kBytes; }
 
-cudaError_t launch_fwd(const FwdParams& p, int d, cudaStream_t stream) {
-    const int BH = p.B * p.H;
-    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
-    const dim3 grid(static_cast<unsigned>(BH) * static_cast<unsigned>(n_pairs));
+cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
+    const long long units = static_cast<long long>(p.B) * p.H * ((p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+    const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
     const int smem = fwd_smem_bytes(d);
+    cudaError_t e;
     if (d == 128) {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
+        if ((e = check_register_split(fa_fwd_kernel<128>)) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+            cudaSuccess)
+            return e;
         fa_fwd_kernel<128><<<grid, kFwdThreads, smem, stream>>>(p);
     } else {
-        cudaError_t e = cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
+        if ((e = check_register_split(fa_fwd_kernel<64>)) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+            cudaSuccess)
+            return e;
         fa_fwd_kernel<64><<<grid, kFwdThreads, smem, stream>>>(p);
     }
     return cudaGetLastError();

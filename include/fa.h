@@ -76,8 +76,8 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /*
  * Workspace bytes fa_backward needs for these sizes: the per-row statistic
- * D [B,H,Lq] (fp32) and an fp32 dQ accumulator [B,H,Lq,d], each 256-byte
- * aligned.  Returns 0 for invalid sizes.
+ * D [B,H,Lq] (fp32), rounded up to 256 bytes.  (dQ is computed in its own
+ * pass, so there is no fp32 dQ accumulator.)  Returns 0 for invalid sizes.
  */
 size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d);
 
