@@ -276,11 +276,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             }
             // P^T = exp2(S^T * scale*log2e - LSE*log2e); causal: key > query + off -> 0
             const bool need_mask = p.causal && (j0 + 127 > i0 + off);
+            const float4* lse4 = reinterpret_cast<const float4*>(lse2);  // broadcast reads, 4 per load
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float v = ex2_approx(fmaf(pr[c], sl2, -lse2[c]));
-                if (need_mask && key > i0 + c + off) v = 0.0f;
-                pr[c] = v;
+            for (int c4 = 0; c4 < 16; ++c4) {
+                const float4 lv = lse4[c4];
+                const float lc[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int c = c4 * 4 + x;
+                    float v = ex2_approx(fmaf(pr[c], sl2, -lc[x]));
+                    if (need_mask && key > i0 + c + off) v = 0.0f;
+                    pr[c] = v;
+                }
             }
             {
                 uint32_t pk[32];
@@ -295,19 +302,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             if (!ok) break;
             tc_fence_after();
             {
+                const float4* d4 = reinterpret_cast<const float4*>(dsum);
                 uint32_t u[32], pk[32];
-                tmem_ld32(tDP, u);
-                tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[c] = pack_bf16x2(pr[2 * c] * (__uint_as_float(u[2 * c]) - dsum[2 * c]),
-                                        pr[2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum[2 * c + 1]));
-                tmem_ld32(tDP + 32, u);
-                tmem_wait_ld();
+                for (int h = 0; h < 2; ++h) {
+                    tmem_ld32(tDP + 32 * h, u);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    pk[16 + c] = pack_bf16x2(pr[32 + 2 * c] * (__uint_as_float(u[2 * c]) - dsum[32 + 2 * c]),
-                                             pr[32 + 2 * c + 1] * (__uint_as_float(u[2 * c + 1]) - dsum[32 + 2 * c + 1]));
+                    for (int c4 = 0; c4 < 8; ++c4) {
+                        const float4 dv = d4[h * 8 + c4];
+                        const int c = h * 32 + c4 * 4;
+                        pk[h * 16 + c4 * 2] = pack_bf16x2(pr[c] * (__uint_as_float(u[c4 * 4]) - dv.x),
+                                                          pr[c + 1] * (__uint_as_float(u[c4 * 4 + 1]) - dv.y));
+                        pk[h * 16 + c4 * 2 + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(u[c4 * 4 + 2]) - dv.z),
+                                                              pr[c + 3] * (__uint_as_float(u[c4 * 4 + 3]) - dv.w));
+                    }
+                }
                 tmem_st32(tDP, pk);
                 tmem_wait_st();
             }

@@ -374,23 +374,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 const float m_new = fmaxf(m_ref, mx);
                 const bool want =
                     (m_ref == -INFINITY) ? (m_new != -INFINITY) : ((m_new - m_ref) * sl2 > kRescaleLog2);
-                if (__any_sync(0xffffffffu, want)) {
-                    const float alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
+                float alpha = 1.0f;
+                const bool rescale = __any_sync(0xffffffffu, want);
+                if (rescale) {
+                    alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
                     l *= alpha;
                     corr *= alpha;
                     m_ref = m_new;
-                    if (j > 0) {
-                        // Small chunks: the score row stays live in registers meanwhile.
-#pragma unroll 1
-                        for (int c = 0; c < D / 8; ++c) {
-                            uint32_t r[8];
-                            tmem_ld8(t_o + c * 8, r);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int x = 0; x < 8; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * alpha);
-                            tmem_st8(t_o + c * 8, r);
-                        }
-                    }
                 }
                 const float mb = (m_ref == -INFINITY) ? 0.0f : m_ref * sl2;
                 uint32_t pk[kFwdBN / 2];
@@ -421,6 +411,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 tmem_st16(t_s + 16, pk + 16);
                 tmem_st16(t_s + 32, pk + 32);
                 tmem_st16(t_s + 48, pk + 48);
+                if (rescale && j > 0) {
+                    // O~ <- alpha O~ for this row (warp-uniform branch).  PV_{j-1} is
+                    // complete: S_j's commit tracked every earlier MMA.  Done after
+                    // P is written so the score registers are free for the row of O.
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {  // 32 columns at a time
+                        uint32_t r0[32];
+                        tmem_ld32(t_o + c * 32, r0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) r0[x] = __float_as_uint(__uint_as_float(r0[x]) * alpha);
+                        tmem_st32(t_o + c * 32, r0);
+                    }
+                }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bar_p[w]);
