@@ -384,21 +384,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 }
                 const float mb = (m_ref == -INFINITY) ? 0.0f : m_ref * sl2;
                 uint32_t pk[kFwdBN / 2];
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};
+                // Packed fp32 pairs (sm_100 FFMA2/FADD2): scale-and-subtract and the row sum.
+                const float2 sl2x2 = make_float2(sl2, sl2);
+                const float2 nmb2 = make_float2(-mb, -mb);
+                float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < kFwdBN; c += 2) {
-                    const float x0 = fmaf(s[c], sl2, -mb);
-                    const float x1 = fmaf(s[c + 1], sl2, -mb);
-                    float p0 = emulated_col(c) ? exp2_poly(x0) : ex2_approx(x0);
-                    float p1 = emulated_col(c + 1) ? exp2_poly(x1) : ex2_approx(x1);
+                    const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2x2, nmb2);
+                    float p0 = emulated_col(c) ? exp2_poly(x.x) : ex2_approx(x.x);
+                    float p1 = emulated_col(c + 1) ? exp2_poly(x.y) : ex2_approx(x.y);
                     if (need_mask) {  // exact zeros for masked keys
                         p0 = (kv0 + c > limit) ? 0.0f : p0;
                         p1 = (kv0 + c + 1 > limit) ? 0.0f : p1;
                     }
-                    ls[(c >> 1) & 3] += p0 + p1;
+                    ls2[(c >> 1) & 1] = __fadd2_rn(ls2[(c >> 1) & 1], make_float2(p0, p1));
                     pk[c >> 1] = pack_bf16x2(p0, p1);
                 }
-                l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+                {
+                    const float2 t = __fadd2_rn(ls2[0], ls2[1]);
+                    l += t.x + t.y;
+                }
                 {
                     // The tile's largest P~ dominates its row's rounding error: account
                     // for its bf16 rounding in the normaliser of O (recomputed on the
