@@ -402,6 +402,50 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
     return legs
 
 
+def run_profile_case(args, device):
+    """One path of the library, W + K calls on seeded device inputs, for a profiler
+    (ncu) to capture; prints a single status line.  fwd: the headline forward;
+    bwd: forward then backward at the 8,192-token training shape; decode_small:
+    decode at B=16 H=32 cap=8192 (1 GiB of cache, small enough to capture)."""
+    import torch
+
+    import exact_io_aware_94_b200 as fa
+    from exact_io_aware_94_b200.inputs import WORKLOADS
+
+    gen = torch.Generator(device=device).manual_seed(11)
+    stream = torch.cuda.current_stream(device)
+    calls = args.warmup + args.steps
+    if args.profile_case in ("fwd", "bwd"):
+        w = WORKLOADS[HEADLINE if args.profile_case == "fwd" else "train_L8192"]
+        B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+        q = (torch.randn(B, H, L, d, generator=gen, device=device) * w["q_scale"]).to(torch.bfloat16)
+        k, v, g = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+        o, lse = fa.forward(q, k, v, causal=True, stream=stream)
+        if args.profile_case == "fwd":
+            for _ in range(calls):
+                fa.forward(q, k, v, causal=True, out=o, lse=lse, stream=stream)
+        else:
+            ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), device)
+            for _ in range(calls):
+                fa.backward(q, k, v, o, g, lse, causal=True, ws=ws, stream=stream)
+        nbytes = 0
+    else:
+        B, H, cap, d = 16, 32, 8192, 128
+        kc, vc = (torch.randn(B, H, cap, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(2))
+        qd = torch.randn(B, H, d, generator=gen, device=device).to(torch.bfloat16)
+        lens = torch.randint(1024, cap + 1, (B,), generator=torch.Generator().manual_seed(5)).to(torch.int32)
+        ws = fa.workspace(fa.fa_decode_workspace_size(B, H, cap, d), device)
+        lens_d = lens.to(device)
+        for _ in range(calls):
+            fa.decode(qd, kc, vc, lens_d, ws=ws, stream=stream)
+        nbytes = int(lens.sum()) * H * d * 2 * 2
+    torch.cuda.synchronize()
+    status = fa.fa_check_status(stream)
+    print(json.dumps({"profile_case": args.profile_case, "calls": calls, "status": status,
+                      "algorithmic_kv_bytes_per_call": nbytes}), flush=True)
+    return 0 if status == fa.FA_OK else 1
+
+
 def run_reference(args, rank):
     """The oracle, as it stands, on the host cores: bounded samples of the same workload."""
     if rank != 0:
@@ -438,9 +482,11 @@ def main(argv=None):
     ap.add_argument("--legs", choices=["all", "none"], default="all")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-budget", type=float, default=8.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small"], default=None,
+                    help="run only this path W+K times for a profiler; no benchmark line")
     args = ap.parse_args(argv)
-    if args.warmup < 3:
+    if args.impl == "ours" and args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -458,6 +504,8 @@ def main(argv=None):
 
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
+    if args.profile_case:
+        return run_profile_case(args, device)
     if world > 1:
         import datetime
 

@@ -25,8 +25,8 @@ constexpr int kBwdThreads = 320;  // 2 elementwise warpgroups + TMA warp + MMA w
 // grow to kFwdRegsSoftmax, the TMA/MMA warpgroup shrinks to kFwdRegsOther.  The
 // launch allocation must cover the split: kFwdThreads x (registers the kernel is
 // compiled with) >= 2*128*kFwdRegsSoftmax + 128*kFwdRegsOther; launch_fwd checks.
-constexpr int kFwdRegsSoftmax = 216;
-constexpr int kFwdRegsOther = 72;
+constexpr int kFwdRegsSoftmax = 200;
+constexpr int kFwdRegsOther = 104;
 
 struct __align__(64) FwdParams {
     CUtensorMap tm_q;  // [B*H, Lq, d] bf16, box {64, 128, 1}, 128B swizzle

@@ -29,8 +29,7 @@
 // The LSE uses the running sum of the unrounded P~.  O is normalised by that
 // sum plus, per tile, the bf16 rounding error of the tile's largest P~ (the
 // term that dominates a peaky row), so numerator and denominator weigh the
-// dominant key alike.  Optionally some exponentials run as a polynomial on the
-// FMA pipe instead of MUFU (off by default, see kEmuPer8).
+// dominant key alike.  P~ is handed to the MMA in two halves of 64 keys.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,15 +42,7 @@ namespace {
 
 constexpr float kRescaleLog2 = 8.0f;
 
-// Of every 8 consecutive score columns, the last kEmuPer8 take their
-// exponential on the FMA pipe (polynomial) instead of MUFU.  Measured on B200
-// the softmax is issue-bound rather than MUFU-bound (every fraction tried
-// from 1/8 to 3/8 was slower), so the default is 0.
-#ifndef FA_FWD_EMU_PER8
-#define FA_FWD_EMU_PER8 0
-#endif
-constexpr int kEmuPer8 = FA_FWD_EMU_PER8;
-__device__ __forceinline__ constexpr bool emulated_col(int c) { return (c & 7) >= 8 - kEmuPer8; }
+
 
 template <int D>
 struct FwdLayout {
@@ -63,8 +54,8 @@ struct FwdLayout {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    // barriers: q, q_free, k[S], v[S], empty[S], s[2], p[2], o[2], o_free[2], drain
-    static constexpr int kNumBars = 2 + 3 * kStages + 2 * 4 + 1;
+    // barriers: q, q_free, k[S], v[S], empty[S], s[2], p[2][2 halves], o[2], o_free[2], drain
+    static constexpr int kNumBars = 2 + 3 * kStages + 10 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16 + 1024;  // + tmem slot/abort + alignment slack
 };
@@ -119,8 +110,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint64_t* bar_v = bars + 2 + S;
     uint64_t* bar_empty = bars + 2 + 2 * S;
     uint64_t* bar_s = bars + 2 + 3 * S;
-    uint64_t* bar_p = bar_s + 2;
-    uint64_t* bar_o = bar_p + 2;
+    uint64_t* bar_p = bar_s + 2;  // [2 * w + half]
+    uint64_t* bar_o = bar_p + 4;
     uint64_t* bar_ofree = bar_o + 2;
     uint64_t* bar_drain = bar_ofree + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
@@ -149,7 +140,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(&bar_s[w], 1);
-            mbar_init(&bar_p[w], 4 * 32);
+            mbar_init(&bar_p[2 * w], 4 * 32);
+            mbar_init(&bar_p[2 * w + 1], 4 * 32);
             mbar_init(&bar_o[w], 1);
             mbar_init(&bar_ofree[w], 4 * 32);
         }
@@ -235,11 +227,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 }
                 umma_commit(&bar_s[w]);
             };
-            auto issue_pv = [&](int w, int s, int j) {
+            // PV for one half of the tile's keys (h = 0: keys 0-63, h = 1: keys 64-127).
+            auto issue_pv_half = [&](int w, int s, int j, int h) {
                 const uint32_t t_p = tmem_base + w * 128;
                 const uint32_t t_o = tmem_base + 256 + w * D;
 #pragma unroll
-                for (int kk = 0; kk < kFwdBN / 16; ++kk) {
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int kk = h * 4 + k4;
                     const uint64_t b =
                         smem_desc_sw128(sVa + s * Lay::kTileBytes + kk * 2048, Lay::kBoxBytes, 1024);
                     umma_ts(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
@@ -275,10 +269,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                                 if (!(ok = mbar_wait(&bar_ofree[w], (units_w[w] - 1) & 1, abort_flag, p.status)))
                                     break;
                             }
-                            if (!(ok = mbar_wait(&bar_p[w], tp[w] & 1, abort_flag, p.status))) break;
+                            if (!(ok = mbar_wait(&bar_p[2 * w], tp[w] & 1, abort_flag, p.status))) break;
+                            tc_fence_after();
+                            issue_pv_half(w, s, j, 0);
+                            if (!(ok = mbar_wait(&bar_p[2 * w + 1], tp[w] & 1, abort_flag, p.status))) break;
                             ++tp[w];
                             tc_fence_after();
-                            issue_pv(w, s, j);
+                            issue_pv_half(w, s, j, 1);
                             if (j == nw - 1) {
                                 umma_commit(&bar_o[w]);
                                 ++units_w[w];
@@ -352,87 +349,76 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     for (int c = 0; c < kFwdBN; ++c)
                         if (kv0 + c > limit) s[c] = -INFINITY;
                 }
-                // Row max, kept separately over the columns whose exponential runs
-                // on MUFU (mx_a) and on the FMA pipe (mx_b), so the rounding
-                // correction below can redo the max element on the same path.
-                float mx_a, mx_b;
+                // Row max: eight independent chains, then a tree.
+                float mx;
                 {
-                    float ma[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                    float mb2[2] = {-INFINITY, -INFINITY};
+                    float ma[8];
 #pragma unroll
-                    for (int c = 0; c < kFwdBN; c += 2) {
-                        if (emulated_col(c)) {
-                            mb2[(c >> 3) & 1] = fmax3(mb2[(c >> 3) & 1], s[c], s[c + 1]);
-                        } else {
-                            ma[(c >> 1) & 3] = fmax3(ma[(c >> 1) & 3], s[c], s[c + 1]);
-                        }
-                    }
-                    mx_a = fmax3(ma[0], ma[1], fmaxf(ma[2], ma[3]));
-                    mx_b = fmaxf(mb2[0], mb2[1]);
+                    for (int x = 0; x < 8; ++x) ma[x] = s[x];
+#pragma unroll
+                    for (int c = 8; c < kFwdBN; ++c) ma[c & 7] = fmaxf(ma[c & 7], s[c]);
+                    mx = fmaxf(fmaxf(fmaxf(ma[0], ma[1]), fmaxf(ma[2], ma[3])),
+                               fmaxf(fmaxf(ma[4], ma[5]), fmaxf(ma[6], ma[7])));
                 }
-                const float mx = fmaxf(mx_a, mx_b);
                 const float m_new = fmaxf(m_ref, mx);
                 const bool want =
                     (m_ref == -INFINITY) ? (m_new != -INFINITY) : ((m_new - m_ref) * sl2 > kRescaleLog2);
-                float alpha = 1.0f;
-                const bool rescale = __any_sync(0xffffffffu, want);
-                if (rescale) {
-                    alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
+                if (__any_sync(0xffffffffu, want)) {
+                    const float alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx((m_ref - m_new) * sl2);
                     l *= alpha;
                     corr *= alpha;
                     m_ref = m_new;
+                    if (j > 0) {
+                        // O~ <- alpha O~ (warp-uniform branch, rare).  PV_{j-1} is complete:
+                        // the commit that signalled S_j tracked every earlier MMA.
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t r0[32];
+                            tmem_ld32(t_o + c * 32, r0);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) r0[x] = __float_as_uint(__uint_as_float(r0[x]) * alpha);
+                            tmem_st32(t_o + c * 32, r0);
+                        }
+                    }
                 }
                 const float mb = (m_ref == -INFINITY) ? 0.0f : m_ref * sl2;
-                uint32_t pk[kFwdBN / 2];
-                // Packed fp32 pairs (sm_100 FFMA2/FADD2): scale-and-subtract and the row sum.
+                // P~ = exp2(s * scale*log2e - m * scale*log2e) in two halves of 64 keys;
+                // each half is handed to the MMA as soon as it is in TMEM, so the
+                // first half of PV runs while the second half is computed.
+                // Packed fp32 pairs (FFMA2/FADD2) for the scale-subtract and the sum.
                 const float2 sl2x2 = make_float2(sl2, sl2);
                 const float2 nmb2 = make_float2(-mb, -mb);
                 float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                for (int c = 0; c < kFwdBN; c += 2) {
-                    const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2x2, nmb2);
-                    float p0 = emulated_col(c) ? exp2_poly(x.x) : ex2_approx(x.x);
-                    float p1 = emulated_col(c + 1) ? exp2_poly(x.y) : ex2_approx(x.y);
-                    if (need_mask) {  // exact zeros for masked keys
-                        p0 = (kv0 + c > limit) ? 0.0f : p0;
-                        p1 = (kv0 + c + 1 > limit) ? 0.0f : p1;
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[kFwdBN / 4];
+#pragma unroll
+                    for (int c = h * 64; c < h * 64 + 64; c += 2) {
+                        const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2x2, nmb2);
+                        float p0 = ex2_approx(x.x);
+                        float p1 = ex2_approx(x.y);
+                        if (need_mask) {  // exact zeros for masked keys
+                            p0 = (kv0 + c > limit) ? 0.0f : p0;
+                            p1 = (kv0 + c + 1 > limit) ? 0.0f : p1;
+                        }
+                        ls2[(c >> 1) & 1] = __fadd2_rn(ls2[(c >> 1) & 1], make_float2(p0, p1));
+                        pk[(c - h * 64) >> 1] = pack_bf16x2(p0, p1);
                     }
-                    ls2[(c >> 1) & 1] = __fadd2_rn(ls2[(c >> 1) & 1], make_float2(p0, p1));
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                    tmem_st16(t_s + h * 32, pk);
+                    tmem_st16(t_s + h * 32 + 16, pk + 16);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&bar_p[2 * w + h]);
                 }
                 {
-                    const float2 t = __fadd2_rn(ls2[0], ls2[1]);
-                    l += t.x + t.y;
-                }
-                {
+                    const float2 t2 = __fadd2_rn(ls2[0], ls2[1]);
+                    l += t2.x + t2.y;
                     // The tile's largest P~ dominates its row's rounding error: account
-                    // for its bf16 rounding in the normaliser of O (recomputed on the
-                    // same exponential path as the element itself).
-                    const float xm = fmaf(mx, sl2, -mb);
-                    const float pmax = (mx == -INFINITY) ? 0.0f : (mx_b > mx_a ? exp2_poly(xm) : ex2_approx(xm));
+                    // for its bf16 rounding in the normaliser of O.
+                    const float pmax = (mx == -INFINITY) ? 0.0f : ex2_approx(fmaf(mx, sl2, -mb));
                     corr += round_bf16(pmax) - pmax;
                 }
-                tmem_st16(t_s + 0, pk + 0);
-                tmem_st16(t_s + 16, pk + 16);
-                tmem_st16(t_s + 32, pk + 32);
-                tmem_st16(t_s + 48, pk + 48);
-                if (rescale && j > 0) {
-                    // O~ <- alpha O~ for this row (warp-uniform branch).  PV_{j-1} is
-                    // complete: S_j's commit tracked every earlier MMA.  Done after
-                    // P is written so the score registers are free for the row of O.
-#pragma unroll 1
-                    for (int c = 0; c < D / 32; ++c) {  // 32 columns at a time
-                        uint32_t r0[32];
-                        tmem_ld32(t_o + c * 32, r0);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) r0[x] = __float_as_uint(__uint_as_float(r0[x]) * alpha);
-                        tmem_st32(t_o + c * 32, r0);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bar_p[w]);
             }
             if (!ok) break;
 
