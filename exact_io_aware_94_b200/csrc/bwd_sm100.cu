@@ -340,16 +340,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
                     uint32_t u[32];
                     tmem_ld32(tmem_base + lane_bits + col0 + c * 32, u);
                     tmem_wait_ld();
-                    if (valid) {
-                        uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+                    if (valid) {  // 32-byte stores
 #pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            uint4 o;
-                            o.x = pack_bf16x2(__uint_as_float(u[8 * x + 0]) * mul, __uint_as_float(u[8 * x + 1]) * mul);
-                            o.y = pack_bf16x2(__uint_as_float(u[8 * x + 2]) * mul, __uint_as_float(u[8 * x + 3]) * mul);
-                            o.z = pack_bf16x2(__uint_as_float(u[8 * x + 4]) * mul, __uint_as_float(u[8 * x + 5]) * mul);
-                            o.w = pack_bf16x2(__uint_as_float(u[8 * x + 6]) * mul, __uint_as_float(u[8 * x + 7]) * mul);
-                            d4[x] = o;
+                        for (int x = 0; x < 2; ++x) {
+                            uint32_t v8[8];
+#pragma unroll
+                            for (int y = 0; y < 8; ++y)
+                                v8[y] = pack_bf16x2(__uint_as_float(u[16 * x + 2 * y]) * mul,
+                                                    __uint_as_float(u[16 * x + 2 * y + 1]) * mul);
+                            st_global_v8(dst + c * 32 + 16 * x, v8);
                         }
                     }
                 }
@@ -605,16 +604,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
                 uint32_t u[32];
                 tmem_ld32(tmem_base + lane_bits + kColDQ + w * (D / 2) + c * 32, u);
                 tmem_wait_ld();
-                if (row_valid) {
-                    uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+                if (row_valid) {  // 32-byte stores
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(u[8 * x + 0]) * p.scale, __uint_as_float(u[8 * x + 1]) * p.scale);
-                        o.y = pack_bf16x2(__uint_as_float(u[8 * x + 2]) * p.scale, __uint_as_float(u[8 * x + 3]) * p.scale);
-                        o.z = pack_bf16x2(__uint_as_float(u[8 * x + 4]) * p.scale, __uint_as_float(u[8 * x + 5]) * p.scale);
-                        o.w = pack_bf16x2(__uint_as_float(u[8 * x + 6]) * p.scale, __uint_as_float(u[8 * x + 7]) * p.scale);
-                        d4[x] = o;
+                    for (int x = 0; x < 2; ++x) {
+                        uint32_t v8[8];
+#pragma unroll
+                        for (int y = 0; y < 8; ++y)
+                            v8[y] = pack_bf16x2(__uint_as_float(u[16 * x + 2 * y]) * p.scale,
+                                                __uint_as_float(u[16 * x + 2 * y + 1]) * p.scale);
+                        st_global_v8(dst + c * 32 + 16 * x, v8);
                     }
                 }
             }

@@ -441,23 +441,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             if (row < p.Lq) {
                 const float inv_l = 1.0f / (l + corr);
                 const size_t row_idx = static_cast<size_t>(un.bh) * p.Lq + row;
+                // 32-byte stores: each fills one sector of the row
                 if (p.o_dtype == FA_DT_F32) {
-                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + row_idx * D);
-#pragma unroll
-                    for (int x = 0; x < D / 4; ++x)
-                        dst[x] = make_float4(__uint_as_float(ov[4 * x]) * inv_l, __uint_as_float(ov[4 * x + 1]) * inv_l,
-                                             __uint_as_float(ov[4 * x + 2]) * inv_l,
-                                             __uint_as_float(ov[4 * x + 3]) * inv_l);
-                } else {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + row_idx * D);
+                    float* dst = static_cast<float*>(p.o) + row_idx * D;
 #pragma unroll
                     for (int x = 0; x < D / 8; ++x) {
-                        uint4 v4;
-                        v4.x = pack_bf16x2(__uint_as_float(ov[8 * x + 0]) * inv_l, __uint_as_float(ov[8 * x + 1]) * inv_l);
-                        v4.y = pack_bf16x2(__uint_as_float(ov[8 * x + 2]) * inv_l, __uint_as_float(ov[8 * x + 3]) * inv_l);
-                        v4.z = pack_bf16x2(__uint_as_float(ov[8 * x + 4]) * inv_l, __uint_as_float(ov[8 * x + 5]) * inv_l);
-                        v4.w = pack_bf16x2(__uint_as_float(ov[8 * x + 6]) * inv_l, __uint_as_float(ov[8 * x + 7]) * inv_l);
-                        dst[x] = v4;
+                        uint32_t v8[8];
+#pragma unroll
+                        for (int y = 0; y < 8; ++y) v8[y] = __float_as_uint(__uint_as_float(ov[8 * x + y]) * inv_l);
+                        st_global_v8(dst + 8 * x, v8);
+                    }
+                } else {
+                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + row_idx * D;
+#pragma unroll
+                    for (int x = 0; x < D / 16; ++x) {
+                        uint32_t v8[8];
+#pragma unroll
+                        for (int y = 0; y < 8; ++y)
+                            v8[y] = pack_bf16x2(__uint_as_float(ov[16 * x + 2 * y]) * inv_l,
+                                                __uint_as_float(ov[16 * x + 2 * y + 1]) * inv_l);
+                        st_global_v8(dst + 16 * x, v8);
                     }
                 }
                 p.lse[row_idx] = m_ref * p.scale + logf(l);
