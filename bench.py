@@ -350,7 +350,8 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
     legs["train_L8192_bwd"] = {"ms": round(t_b * 1e3, 4), "TFLOP/s": round(fb / t_b / 1e12, 1),
                                "frac_of_peak": round(fb / t_b / 1e12 / peaks["bf16_tflops"], 4),
                                "launches": 3, "kernels": "fa_bwd_dot + fa_bwd_dkdv + fa_bwd_dq",
-                               "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 7"}
+                               "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 7",
+                               "traffic": recorded_traffic("fa_bwd", "train_L8192", ["bwd_sm100.cu", "ptx.cuh"])}
     del q, k, v, g, o, lse, dq, dk, dv, ws
 
     # 65,536-token forward
@@ -394,7 +395,8 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "frac_of_peak": round(nbytes / t_d / 1e9 / peaks["hbm_gbs"], 4),
                                "frac_of_nominal_8000": round(nbytes / t_d / 1e9 / NOMINAL_HBM_GBS, 4),
                                "launches": 3, "kernels": "fa_decode_plan + fa_decode_split + fa_decode_combine",
-                               "l2": "caches 2 x 16 GiB, far larger than L2"}
+                               "l2": "caches 2 x 16 GiB, far larger than L2",
+                               "traffic": recorded_traffic("fa_decode", "decode_cap32768", ["decode_sm100.cu"])}
     del kc, vc
     status = fa.fa_check_status(stream)
     if status != fa.FA_OK:
