@@ -194,55 +194,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             for (int t = max(0, issued - S); t < issued; ++t) mbar_wait_drain(&bar_qd[t % S], (t / S) & 1, p.status);
         }
     } else if (warp == 9) {
-        // ================= MMA issuer
-        if (lane == 0) {
+        // ================= MMA issuer: the whole warp runs the loop (operands stay
+        // warp-uniform), one lane chosen by elect.sync issues each MMA and commit
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        {
             constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sGa = smem_u32(sG);
-            bool ok = mbar_wait(bar_kv, 0, abort_flag, p.status);
+            bool ok = wait(bar_kv, 0);
             for (int t = 0; ok && t < nq; ++t) {
                 const int s = t % S;
-                if (!(ok = mbar_wait(&bar_qd[s], (t / S) & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(&bar_qd[s], (t / S) & 1))) break;
                 tc_fence_after();
                 // S^T = K Q^T, dP^T = V dO^T   (M = 128 keys, N = 128 queries, K = D)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
-                    umma_ss(tmem_base + kColS, smem_desc_sw128(sKa + koff, 16, 1024),
+                    umma_ss_w(tmem_base + kColS, smem_desc_sw128(sKa + koff, 16, 1024),
                             smem_desc_sw128(sQa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
-                umma_commit(bar_s);
+                umma_commit_w(bar_s);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
-                    umma_ss(tmem_base + kColDP, smem_desc_sw128(sVa + koff, 16, 1024),
+                    umma_ss_w(tmem_base + kColDP, smem_desc_sw128(sVa + koff, 16, 1024),
                             smem_desc_sw128(sGa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
-                umma_commit(bar_dp);
+                umma_commit_w(bar_dp);
                 // dV += P^T dO   (A = P^T from TMEM: queries 0-63 at cols [0,32), 64-127 at [64,96))
-                if (!(ok = mbar_wait(bar_p, t & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(bar_p, t & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem_base + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_ts(tmem_base + kColDV, a,
+                    umma_ts_w(tmem_base + kColDV, a,
                             smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 // dK += dS^T Q
-                if (!(ok = mbar_wait(bar_ds, t & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(bar_ds, t & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem_base + kColDP + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_ts(tmem_base + kColDK, a,
+                    umma_ts_w(tmem_base + kColDK, a,
                             smem_desc_sw128(sQa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
                             (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bar_empty[s]);
+                umma_commit_w(&bar_empty[s]);
             }
-            if (ok) umma_commit(bar_acc);
-            umma_commit(bar_drain);
+            if (ok) umma_commit_w(bar_acc);
+            umma_commit_w(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.status);
         }
     } else {
@@ -443,24 +447,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 8) {
-        if (lane == 0 && !*abort_flag) {
-            tma_prefetch_desc(&p.tm_k);
-            tma_prefetch_desc(&p.tm_v);
-            mbar_arrive_expect_tx(bar_qd, 2 * T::kTileBytes);
+        // producer: whole warp, one elected lane issues each copy
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        if (!*abort_flag) {
+            if (lane == 0) {
+                tma_prefetch_desc(&p.tm_k);
+                tma_prefetch_desc(&p.tm_v);
+            }
+            mbar_arrive_expect_tx_w(bar_qd, 2 * T::kTileBytes);
             for (int b = 0; b < T::kBoxes; ++b) {
-                tma_load_3d(sQ + b * T::kBoxBytes, &p.tm_q, bar_qd, b * 64, i0, bh);
-                tma_load_3d(sG + b * T::kBoxBytes, &p.tm_do, bar_qd, b * 64, i0, bh);
+                tma_load_3d_w(sQ + b * T::kBoxBytes, &p.tm_q, bar_qd, b * 64, i0, bh);
+                tma_load_3d_w(sG + b * T::kBoxBytes, &p.tm_do, bar_qd, b * 64, i0, bh);
             }
             int issued = 0;
             for (int j = 0; j < nk; ++j) {
                 const int s = j % S;
-                if (j >= S && !mbar_wait(&bar_empty[s], ((j / S) - 1) & 1, abort_flag, p.status)) break;
-                mbar_arrive_expect_tx(&bar_k[s], T::kTileBytes);
+                if (j >= S && !wait(&bar_empty[s], ((j / S) - 1) & 1)) break;
+                mbar_arrive_expect_tx_w(&bar_k[s], T::kTileBytes);
                 for (int b = 0; b < T::kBoxes; ++b)
-                    tma_load_3d(sK + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_k, &bar_k[s], b * 64, j * 128, bh);
-                mbar_arrive_expect_tx(&bar_v[s], T::kTileBytes);
+                    tma_load_3d_w(sK + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_k, &bar_k[s], b * 64, j * 128, bh);
+                mbar_arrive_expect_tx_w(&bar_v[s], T::kTileBytes);
                 for (int b = 0; b < T::kBoxes; ++b)
-                    tma_load_3d(sV + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_v, &bar_v[s], b * 64, j * 128, bh);
+                    tma_load_3d_w(sV + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_v, &bar_v[s], b * 64, j * 128, bh);
                 issued = j + 1;
             }
             if (*abort_flag) {
@@ -472,7 +482,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
             }
         }
     } else if (warp == 9) {
-        if (lane == 0) {
+        // MMA issuer: whole warp, one elected lane issues (see the dK/dV kernel)
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        {
             constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sQa = smem_u32(sQ), sGa = smem_u32(sG), sKa = smem_u32(sK), sVa = smem_u32(sV);
@@ -481,26 +495,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
-                    umma_ss(tmem_base + (j & 1) * 128, smem_desc_sw128(sQa + koff, 16, 1024),
+                    umma_ss_w(tmem_base + (j & 1) * 128, smem_desc_sw128(sQa + koff, 16, 1024),
                             smem_desc_sw128(sKa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
-                umma_commit(&bar_s[j & 1]);
+                umma_commit_w(&bar_s[j & 1]);
             };
             auto issue_dp = [&](int j) {
                 const int s = j % S;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
-                    umma_ss(tmem_base + kColDP, smem_desc_sw128(sGa + koff, 16, 1024),
+                    umma_ss_w(tmem_base + kColDP, smem_desc_sw128(sGa + koff, 16, 1024),
                             smem_desc_sw128(sVa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
-                umma_commit(bar_dp);
+                umma_commit_w(bar_dp);
             };
-            bool ok = mbar_wait(bar_qd, 0, abort_flag, p.status) && mbar_wait(&bar_k[0], 0, abort_flag, p.status);
+            bool ok = wait(bar_qd, 0) && wait(&bar_k[0], 0);
             if (ok) {
                 tc_fence_after();
                 issue_s(0);
-                ok = mbar_wait(&bar_v[0], 0, abort_flag, p.status);
+                ok = wait(&bar_v[0], 0);
                 if (ok) {
                     tc_fence_after();
                     issue_dp(0);
@@ -509,29 +523,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
             for (int j = 0; ok && j < nk; ++j) {
                 const int s = j % S, s1 = (j + 1) % S;
                 if (j + 1 < nk) {
-                    if (!(ok = mbar_wait(&bar_k[s1], ((j + 1) / S) & 1, abort_flag, p.status))) break;
+                    if (!(ok = wait(&bar_k[s1], ((j + 1) / S) & 1))) break;
                     tc_fence_after();
                     issue_s(j + 1);
                 }
                 // dS_j ready in S buffer j&1 (and dP_j read): dQ += dS_j K_j
-                if (!(ok = mbar_wait(bar_dsr, j & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(bar_dsr, j & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem_base + (j & 1) * 128 + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_ts(tmem_base + kColDQ, a,
+                    umma_ts_w(tmem_base + kColDQ, a,
                             smem_desc_sw128(sKa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bar_empty[s]);
+                umma_commit_w(&bar_empty[s]);
                 if (j + 1 < nk) {
-                    if (!(ok = mbar_wait(&bar_v[s1], ((j + 1) / S) & 1, abort_flag, p.status))) break;
+                    if (!(ok = wait(&bar_v[s1], ((j + 1) / S) & 1))) break;
                     tc_fence_after();
                     issue_dp(j + 1);
                 }
             }
-            if (ok) umma_commit(bar_acc);
-            umma_commit(bar_drain);
+            if (ok) umma_commit_w(bar_acc);
+            umma_commit_w(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.status);
         }
     } else {

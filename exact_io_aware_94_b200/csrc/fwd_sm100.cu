@@ -12,8 +12,12 @@
 // the current unit's last S MMA has been issued, so loads, MMAs and the
 // epilogue of consecutive units overlap.
 //   warp 8      TMA producer: Q tiles per unit, K_j / V_j through a smem ring.
-//   warp 9      MMA issuer (one thread): S_w = Q_w K_j^T into TMEM (SS MMA),
+//   warp 9      MMA issuer: S_w = Q_w K_j^T into TMEM (SS MMA),
 //               O_w += P_w V_j with P_w read from TMEM (TS MMA).
+//               In both warps the whole warp runs the control flow and one
+//               lane chosen by elect.sync issues each copy or MMA: the
+//               operands then stay warp-uniform, which keeps the issue cost
+//               per MMA well under the MMA's own 64 cycles.
 //   warps 10-11 idle (they complete the third warpgroup, whose registers
 //               setmaxnreg hands to the softmax warpgroups).
 //   warps 0-3   softmax warpgroup 0 (rows 0..127 of the unit), warps 4-7
@@ -170,7 +174,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
     if (warp == 8) {
         // ================= TMA producer =================
-        if (lane == 0 && !*abort_flag) {
+        // The whole warp runs the loop; one elected lane issues each copy.
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        if (!*abort_flag) {
             int kc = 0;       // K/V tiles issued so far (ring position)
             int q_iter = 0;   // units whose Q has been requested
             bool ok = true;
@@ -178,26 +186,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 const Unit un = unit_of(p, u);
                 const int n_max = max(un.n_kv0, un.n_kv1);
                 // the previous unit's S MMAs must be done with the Q buffer
-                if (q_iter > 0 && !(ok = mbar_wait(bar_q_free, (q_iter - 1) & 1, abort_flag, p.status))) break;
+                if (q_iter > 0 && !(ok = wait(bar_q_free, (q_iter - 1) & 1))) break;
                 const uint32_t q_bytes = (un.n_kv1 > 0 ? 2 : 1) * Lay::kTileBytes;
-                mbar_arrive_expect_tx(bar_q, q_bytes);
+                mbar_arrive_expect_tx_w(bar_q, q_bytes);
                 for (int w = 0; w < 2; ++w) {
                     if ((w == 0 ? un.n_kv0 : un.n_kv1) == 0) continue;
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, bar_q, b * 64,
+                        tma_load_3d_w(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, bar_q, b * 64,
                                     un.i0 + w * kFwdBM, un.bh);
                 }
                 ++q_iter;
                 for (int j = 0; j < n_max; ++j, ++kc) {
                     const int s = kc % S;
-                    if (kc >= S && !(ok = mbar_wait(&bar_empty[s], ((kc / S) - 1) & 1, abort_flag, p.status))) break;
-                    mbar_arrive_expect_tx(&bar_k[s], Lay::kTileBytes);
+                    if (kc >= S && !(ok = wait(&bar_empty[s], ((kc / S) - 1) & 1))) break;
+                    mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
+                        tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
                                     j * kFwdBN, un.bh);
-                    mbar_arrive_expect_tx(&bar_v[s], Lay::kTileBytes);
+                    mbar_arrive_expect_tx_w(&bar_v[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
+                        tma_load_3d_w(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
                                     j * kFwdBN, un.bh);
                 }
             }
@@ -212,7 +220,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         }
     } else if (warp == 9) {
         // ================= MMA issuer =================
-        if (lane == 0) {
+        // The whole warp runs the loop, so descriptors and TMEM addresses are
+        // warp-uniform; one elected lane issues each MMA and commit.
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        {
             constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
@@ -223,9 +236,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     const uint32_t koff = (kk >> 2) * Lay::kBoxBytes + (kk & 3) * 32;
                     const uint64_t a = smem_desc_sw128(sQa + w * Lay::kTileBytes + koff, 16, 1024);
                     const uint64_t b = smem_desc_sw128(sKa + s * Lay::kTileBytes + koff, 16, 1024);
-                    umma_ss(t_s, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+                    umma_ss_w(t_s, a, b, kIdescQK, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&bar_s[w]);
+                umma_commit_w(&bar_s[w]);
             };
             // PV for one half of the tile's keys (h = 0: keys 0-63, h = 1: keys 64-127).
             auto issue_pv_half = [&](int w, int s, int j, int h) {
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     const int kk = h * 4 + k4;
                     const uint64_t b =
                         smem_desc_sw128(sVa + s * Lay::kTileBytes + kk * 2048, Lay::kBoxBytes, 1024);
-                    umma_ts(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts_w(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
             int kc = 0;               // K/V ring position
@@ -248,17 +261,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 const Unit un = unit_of(p, u);
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
-                if (!(ok = mbar_wait(bar_q, q_iter & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(bar_q, q_iter & 1))) break;
                 ++q_iter;
-                if (!(ok = mbar_wait(&bar_k[kc % S], (kc / S) & 1, abort_flag, p.status))) break;
+                if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
                 tc_fence_after();
                 issue_s(0, kc % S);
                 if (n1 > 0) issue_s(1, kc % S);
-                if (n_max == 1) umma_commit(bar_q_free);
+                if (n_max == 1) umma_commit_w(bar_q_free);
                 for (int j = 0; ok && j < n_max; ++j) {
                     const int s = (kc + j) % S;
                     const int s1 = (kc + j + 1) % S;
-                    if (!(ok = mbar_wait(&bar_v[s], ((kc + j) / S) & 1, abort_flag, p.status))) break;
+                    if (!(ok = wait(&bar_v[s], ((kc + j) / S) & 1))) break;
                     bool k_ready = false;
 #pragma unroll
                     for (int w = 0; w < 2; ++w) {
@@ -266,24 +279,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                         if (j < nw) {
                             if (j == 0 && units_w[w] > 0) {
                                 // O_w still holds the previous unit until its epilogue has read it
-                                if (!(ok = mbar_wait(&bar_ofree[w], (units_w[w] - 1) & 1, abort_flag, p.status)))
+                                if (!(ok = wait(&bar_ofree[w], (units_w[w] - 1) & 1)))
                                     break;
                             }
-                            if (!(ok = mbar_wait(&bar_p[2 * w], tp[w] & 1, abort_flag, p.status))) break;
+                            if (!(ok = wait(&bar_p[2 * w], tp[w] & 1))) break;
                             tc_fence_after();
                             issue_pv_half(w, s, j, 0);
-                            if (!(ok = mbar_wait(&bar_p[2 * w + 1], tp[w] & 1, abort_flag, p.status))) break;
+                            if (!(ok = wait(&bar_p[2 * w + 1], tp[w] & 1))) break;
                             ++tp[w];
                             tc_fence_after();
                             issue_pv_half(w, s, j, 1);
                             if (j == nw - 1) {
-                                umma_commit(&bar_o[w]);
+                                umma_commit_w(&bar_o[w]);
                                 ++units_w[w];
                             }
                         }
                         if (j + 1 < nw) {
                             if (!k_ready) {
-                                if (!(ok = mbar_wait(&bar_k[s1], ((kc + j + 1) / S) & 1, abort_flag, p.status)))
+                                if (!(ok = wait(&bar_k[s1], ((kc + j + 1) / S) & 1)))
                                     break;
                                 tc_fence_after();
                                 k_ready = true;
@@ -292,13 +305,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                         }
                     }
                     if (!ok) break;
-                    if (j + 2 == n_max) umma_commit(bar_q_free);  // last S of this unit issued
-                    umma_commit(&bar_empty[s]);
+                    if (j + 2 == n_max) umma_commit_w(bar_q_free);  // last S of this unit issued
+                    umma_commit_w(&bar_empty[s]);
                 }
                 kc += n_max;
             }
             // Drain: every MMA issued by this thread completes before TMEM is freed.
-            umma_commit(bar_drain);
+            umma_commit_w(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.status);
         }
     } else if (warp < 8) {
