@@ -409,12 +409,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 #pragma unroll
                     for (int c = h * 64; c < h * 64 + 64; c += 2) {
                         const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2x2, nmb2);
-                        float p0 = ex2_approx(x.x);
-                        float p1 = ex2_approx(x.y);
-                        if (need_mask) {  // exact zeros for masked keys
-                            p0 = (kv0 + c > limit) ? 0.0f : p0;
-                            p1 = (kv0 + c + 1 > limit) ? 0.0f : p1;
-                        }
+                        // Masked keys hold s = -inf, so x = -inf and ex2 gives exactly +0:
+                        // no select is needed (and none keeps a second copy of this loop).
+                        const float p0 = ex2_approx(x.x);
+                        const float p1 = ex2_approx(x.y);
                         ls2[(c >> 1) & 1] = __fadd2_rn(ls2[(c >> 1) & 1], make_float2(p0, p1));
                         pk[(c - h * 64) >> 1] = pack_bf16x2(p0, p1);
                     }
