@@ -79,6 +79,21 @@ int encode_rows_map(CUtensorMap* map, const void* base, int BH, int L, int d, in
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// O written by TMA stores: [BH, L, d] in fp32 or bf16, boxes of 32 rows x
+// 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzle.  Rows past L are
+// clipped by the copy engine.
+int encode_out_map_impl(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype) {
+    const int esz = o_dtype == FA_DT_F32 ? 4 : 2;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz, static_cast<cuuint64_t>(L) * d * esz};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, o_dtype == FA_DT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 bool dims_ok(int B, int H, int L, int d) {
     if (B <= 0 || H <= 0 || L <= 0) return false;
     const long long bh = static_cast<long long>(B) * H;
@@ -100,6 +115,9 @@ int encode_tile_map(CUtensorMap* map, const void* base, int BH, int L, int d, in
     return encode_rows_map(map, base, BH, L, d, box_rows);
 }
 bool shape_ok(int B, int H, int L, int d) { return dims_ok(B, H, L, d); }
+int encode_out_map(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype) {
+    return encode_out_map_impl(map, base, BH, L, d, o_dtype);
+}
 
 }  // namespace fa
 
@@ -145,6 +163,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, kFwdBM)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    if ((rc = encode_out_map_impl(&p.tm_o, o, BH, Lq, d, o_dtype)) != FA_OK) return rc;
     p.o = o;
     p.lse = lse;
     p.status = st->status_ptr;

@@ -32,6 +32,7 @@ struct __align__(64) FwdParams {
     CUtensorMap tm_q;  // [B*H, Lq, d] bf16, box {64, 128, 1}, 128B swizzle
     CUtensorMap tm_k;  // [B*H, Lk, d]
     CUtensorMap tm_v;  // [B*H, Lk, d]
+    CUtensorMap tm_o;  // O as [B*H, Lq, d] (fp32 or bf16), box {128 bytes, 32 rows, 1}, 128B swizzle
     void* o;
     float* lse;
     int* status;
@@ -97,5 +98,6 @@ cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_
 
 int fwd_smem_bytes(int d);
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
+int encode_out_map(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype);
 
 }  // namespace fa

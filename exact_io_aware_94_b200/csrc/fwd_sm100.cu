@@ -61,7 +61,10 @@ struct FwdLayout {
     // barriers: q, q_free, k[S], v[S], empty[S], s[2], p[2][2 halves], o[2], o_free[2], drain
     static constexpr int kNumBars = 2 + 3 * kStages + 10 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kBytes = kMiscOff + 16 + 1024;  // + tmem slot/abort + alignment slack
+    // epilogue staging for the O tile stores: 4 KB per softmax warp (32 rows x 128 bytes,
+    // 128-byte swizzle, so 1024-byte aligned)
+    static constexpr int kStageOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
+    static constexpr int kBytes = kStageOff + 8 * 4096 + 1024;  // + alignment slack
 };
 
 // One work unit: which (b*H + h), which pair of 128-row tiles, how many KV tiles each needs.
@@ -449,36 +452,55 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bar_ofree[w]);  // O_w may now be overwritten by the next unit's PV
-            if (row < p.Lq) {
+            {
+                // O leaves through the copy engine: per 128-byte column chunk, each
+                // thread writes its row's 128 bytes into the warp's 32-row stage in
+                // the 128-byte-swizzled layout of the O tensor map (16-byte pieces
+                // XOR row % 8: no bank conflicts), and one lane issues the tile store.
+                // Rows past Lq are clipped by the copy engine.
                 const float inv_l = 1.0f / (l + corr);
-                const size_t row_idx = static_cast<size_t>(un.bh) * p.Lq + row;
-                // 32-byte stores: each fills one sector of the row
-                if (p.o_dtype == FA_DT_F32) {
-                    float* dst = static_cast<float*>(p.o) + row_idx * D;
+                uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
+                const bool f32 = p.o_dtype == FA_DT_F32;
+                const int n_chunks = f32 ? D / 32 : D / 64;
 #pragma unroll
-                    for (int x = 0; x < D / 8; ++x) {
-                        uint32_t v8[8];
+                for (int k = 0; k < D / 32; ++k) {
+                    if (k >= n_chunks) break;
+                    // the stage's previous tile store has finished reading it
+                    if (lane == 0) bulk_wait_group_read0();
+                    __syncwarp();
 #pragma unroll
-                        for (int y = 0; y < 8; ++y) v8[y] = __float_as_uint(__uint_as_float(ov[8 * x + y]) * inv_l);
-                        st_global_v8(dst + 8 * x, v8);
+                    for (int q = 0; q < 8; ++q) {
+                        uint4 v;
+                        if (f32) {
+                            const int c0 = k * 32 + q * 4;
+                            v.x = __float_as_uint(__uint_as_float(ov[c0 + 0]) * inv_l);
+                            v.y = __float_as_uint(__uint_as_float(ov[c0 + 1]) * inv_l);
+                            v.z = __float_as_uint(__uint_as_float(ov[c0 + 2]) * inv_l);
+                            v.w = __float_as_uint(__uint_as_float(ov[c0 + 3]) * inv_l);
+                        } else {
+                            const int c0 = (k * 64 + q * 8) & (D - 1);
+                            v.x = pack_bf16x2(__uint_as_float(ov[c0 + 0]) * inv_l, __uint_as_float(ov[c0 + 1]) * inv_l);
+                            v.y = pack_bf16x2(__uint_as_float(ov[c0 + 2]) * inv_l, __uint_as_float(ov[c0 + 3]) * inv_l);
+                            v.z = pack_bf16x2(__uint_as_float(ov[c0 + 4]) * inv_l, __uint_as_float(ov[c0 + 5]) * inv_l);
+                            v.w = pack_bf16x2(__uint_as_float(ov[c0 + 6]) * inv_l, __uint_as_float(ov[c0 + 7]) * inv_l);
+                        }
+                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
                     }
-                } else {
-                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(p.o) + row_idx * D;
-#pragma unroll
-                    for (int x = 0; x < D / 16; ++x) {
-                        uint32_t v8[8];
-#pragma unroll
-                        for (int y = 0; y < 8; ++y)
-                            v8[y] = pack_bf16x2(__uint_as_float(ov[16 * x + 2 * y]) * inv_l,
-                                                __uint_as_float(ov[16 * x + 2 * y + 1]) * inv_l);
-                        st_global_v8(dst + 16 * x, v8);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (tile_first_row + wq * 32 < p.Lq)
+                            tma_store_3d(&p.tm_o, stg, k * (f32 ? 32 : 64), tile_first_row + wq * 32, un.bh);
+                        bulk_commit_group();
                     }
                 }
-                p.lse[row_idx] = m_ref * p.scale + logf(l);
+                if (row < p.Lq) p.lse[static_cast<size_t>(un.bh) * p.Lq + row] = m_ref * p.scale + logf(l);
             }
         }
     }
 
+    // O tile stores issued by this thread are complete before the CTA exits.
+    if (warp < 8 && lane == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     if (warp == 9) {
