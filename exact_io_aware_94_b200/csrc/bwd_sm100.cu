@@ -278,20 +278,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
                 for (int x = 0; x < 32; ++x) pr[32 + x] = __uint_as_float(u[x]);
                 tmem_wait_ld();
             }
-            // P^T = exp2(S^T * scale*log2e - LSE*log2e); causal: key > query + off -> 0
-            const bool need_mask = p.causal && (j0 + 127 > i0 + off);
+            // P^T = exp2(S^T * scale*log2e - LSE*log2e); causal: key > query + off -> 0.
+            // Masked scores are set to -inf first, so the exponential gives exactly +0
+            // with no select in its loop (the LSE of a valid row is finite; rows past
+            // Lq carry +inf).
+            if (p.causal && (j0 + 127 > i0 + off)) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (key > i0 + c + off) pr[c] = -INFINITY;
+            }
             const float4* lse4 = reinterpret_cast<const float4*>(lse2);  // broadcast reads, 4 per load
 #pragma unroll
             for (int c4 = 0; c4 < 16; ++c4) {
                 const float4 lv = lse4[c4];
                 const float lc[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const int c = c4 * 4 + x;
-                    float v = ex2_approx(fmaf(pr[c], sl2, -lc[x]));
-                    if (need_mask && key > i0 + c + off) v = 0.0f;
-                    pr[c] = v;
-                }
+                for (int x = 0; x < 4; ++x) pr[c4 * 4 + x] = ex2_approx(fmaf(pr[c4 * 4 + x], sl2, -lc[x]));
             }
             {
                 uint32_t pk[32];
@@ -578,13 +580,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
                 for (int x = 0; x < 32; ++x) pr[32 + x] = __uint_as_float(u[x]);
                 tmem_wait_ld();
             }
-            const bool need_mask = k0 + 63 > i0 + off || k0 + 64 > p.Lk;
+            // Masked keys (causal, or past Lk) become -inf before the exponential,
+            // which then gives exactly +0 with no select in its loop.
+            if (k0 + 63 > i0 + off || k0 + 64 > p.Lk) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float v = ex2_approx(fmaf(pr[c], sl2, -lse2));
-                if (need_mask && k0 + c > limit) v = 0.0f;
-                pr[c] = v;
+                for (int c = 0; c < 64; ++c)
+                    if (k0 + c > limit) pr[c] = -INFINITY;
             }
+#pragma unroll
+            for (int c = 0; c < 64; ++c) pr[c] = ex2_approx(fmaf(pr[c], sl2, -lse2));
             ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, j & 1, abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
