@@ -8,9 +8,11 @@
 //
 // B200 mapping.  A work unit is 256 query rows of one (b, h): two 128-row Q
 // tiles, one per softmax warpgroup.  The kernel is persistent (one CTA per SM)
-// and walks a static, balanced share of the units; the next unit's Q is loaded as soon as
-// the current unit's last S MMA has been issued, so loads, MMAs and the
-// epilogue of consecutive units overlap.
+// and walks a static, balanced share of the units.  Each warpgroup's Q tile of
+// the next unit is loaded as soon as that warpgroup's last S MMA of the current
+// unit is done with the buffer, and a K slot is refilled once its S MMAs are
+// done (a V slot once its PV MMAs are), so loads, MMAs and the epilogue of
+// consecutive units overlap.
 //   warp 8      TMA producer: Q tiles per unit, K_j / V_j through a smem ring.
 //   warp 9      MMA issuer: S_w = Q_w K_j^T into TMEM (SS MMA),
 //               O_w += P_w V_j with P_w read from TMEM (TS MMA).
@@ -58,8 +60,8 @@ struct FwdLayout {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    // barriers: q, q_free, k[S], v[S], empty[S], s[2], p[2][2 halves], o[2], o_free[2], drain
-    static constexpr int kNumBars = 2 + 3 * kStages + 10 + 1;
+    // barriers: q[2], q_free[2], k[S], v[S], k_free[S], v_free[S], s[2], p[2][2 halves], o[2], o_free[2], drain
+    static constexpr int kNumBars = 4 + 4 * kStages + 10 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // epilogue staging for the O tile stores: 4 KB per softmax warp (32 rows x 128 bytes,
     // 128-byte swizzle, so 1024-byte aligned)
@@ -111,12 +113,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint8_t* sK = smem + Lay::kKOff;
     uint8_t* sV = smem + Lay::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
-    uint64_t* bar_q = bars;
-    uint64_t* bar_q_free = bars + 1;
-    uint64_t* bar_k = bars + 2;
-    uint64_t* bar_v = bars + 2 + S;
-    uint64_t* bar_empty = bars + 2 + 2 * S;
-    uint64_t* bar_s = bars + 2 + 3 * S;
+    uint64_t* bar_q = bars;           // [w]: Q_w landed
+    uint64_t* bar_q_free = bars + 2;  // [w]: the S MMAs of warpgroup w's unit are done with Q_w
+    uint64_t* bar_k = bars + 4;
+    uint64_t* bar_v = bars + 4 + S;
+    // A K slot is free once the S MMAs that read it are done, a V slot once the
+    // PV MMAs are: K runs a tile further ahead than V.
+    uint64_t* bar_kfree = bars + 4 + 2 * S;
+    uint64_t* bar_vfree = bars + 4 + 3 * S;
+    uint64_t* bar_s = bars + 4 + 4 * S;
     uint64_t* bar_p = bar_s + 2;  // [2 * w + half]
     uint64_t* bar_o = bar_p + 4;
     uint64_t* bar_ofree = bar_o + 2;
@@ -138,12 +143,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 
     // ---- setup
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
-        mbar_init(bar_q_free, 1);
+        for (int w = 0; w < 2; ++w) {
+            mbar_init(&bar_q[w], 1);
+            mbar_init(&bar_q_free[w], 1);
+        }
         for (int s = 0; s < S; ++s) {
             mbar_init(&bar_k[s], 1);
             mbar_init(&bar_v[s], 1);
-            mbar_init(&bar_empty[s], 1);
+            mbar_init(&bar_kfree[s], 1);
+            mbar_init(&bar_vfree[s], 1);
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(&bar_s[w], 1);
@@ -182,43 +190,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
         };
         if (!*abort_flag) {
-            int kc = 0;       // K/V tiles issued so far (ring position)
-            int q_iter = 0;   // units whose Q has been requested
+            int kc = 0;                // K/V tiles started so far (ring position)
+            int nk = 0, nv = 0;        // K and V tiles whose loads were issued
+            int q_iter[2] = {0, 0};    // Q tiles requested per warpgroup
             bool ok = true;
             for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
                 const Unit un = unit_of(p, u);
                 const int n_max = max(un.n_kv0, un.n_kv1);
-                // the previous unit's S MMAs must be done with the Q buffer
-                if (q_iter > 0 && !(ok = wait(bar_q_free, (q_iter - 1) & 1))) break;
-                const uint32_t q_bytes = (un.n_kv1 > 0 ? 2 : 1) * Lay::kTileBytes;
-                mbar_arrive_expect_tx_w(bar_q, q_bytes);
-                for (int w = 0; w < 2; ++w) {
-                    if ((w == 0 ? un.n_kv0 : un.n_kv1) == 0) continue;
+                // Q_w as soon as warpgroup w's S MMAs of its previous unit are done with the
+                // buffer (under a causal mask warpgroup 0 lets go of it a tile earlier).
+                // Order Q_0, K_0, Q_1, V_0, K_1, ...
+                auto load_q = [&](int w) -> bool {
+                    if (q_iter[w] > 0 && !wait(&bar_q_free[w], (q_iter[w] - 1) & 1)) return false;
+                    mbar_arrive_expect_tx_w(&bar_q[w], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d_w(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, bar_q, b * 64,
-                                    un.i0 + w * kFwdBM, un.bh);
-                }
-                ++q_iter;
+                        tma_load_3d_w(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, &bar_q[w], b * 64,
+                                      un.i0 + w * kFwdBM, un.bh);
+                    ++q_iter[w];
+                    return true;
+                };
+                if (!(ok = load_q(0))) break;
                 for (int j = 0; j < n_max; ++j, ++kc) {
                     const int s = kc % S;
-                    if (kc >= S && !(ok = wait(&bar_empty[s], ((kc / S) - 1) & 1))) break;
+                    if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
                     mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
                         tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
                                     j * kFwdBN, un.bh);
+                    ++nk;
+                    if (j == 0 && un.n_kv1 > 0 && !(ok = load_q(1))) break;
+                    if (kc >= S && !(ok = wait(&bar_vfree[s], ((kc / S) - 1) & 1))) break;
                     mbar_arrive_expect_tx_w(&bar_v[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
                         tma_load_3d_w(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
                                     j * kFwdBN, un.bh);
+                    ++nv;
                 }
             }
             if (*abort_flag) {
                 // Let copies already in flight land before the CTA's smem goes away.
-                if (q_iter > 0) mbar_wait_drain(bar_q, (q_iter - 1) & 1, p.status);
-                for (int t = max(0, kc - S); t < kc; ++t) {
-                    mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
-                    mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
-                }
+                for (int w = 0; w < 2; ++w)
+                    if (q_iter[w] > 0) mbar_wait_drain(&bar_q[w], (q_iter[w] - 1) & 1, p.status);
+                for (int t = max(0, nk - S); t < nk; ++t) mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
+                for (int t = max(0, nv - S); t < nv; ++t) mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
             }
         }
     } else if (warp == 9) {
@@ -255,22 +269,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     umma_ts_w(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
                 }
             };
-            int kc = 0;               // K/V ring position
-            int q_iter = 0;           // units started
-            int tp[2] = {0, 0};       // P tiles consumed per warpgroup
-            int units_w[2] = {0, 0};  // units whose O_w was handed to the epilogue
+            int kc = 0;                // K/V ring position
+            int q_iter[2] = {0, 0};    // Q tiles consumed per warpgroup
+            int tp[2] = {0, 0};        // P tiles consumed per warpgroup
+            int units_w[2] = {0, 0};   // units whose O_w was handed to the epilogue
             bool ok = true;
             for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
                 const Unit un = unit_of(p, u);
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
-                if (!(ok = wait(bar_q, q_iter & 1))) break;
-                ++q_iter;
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
                 tc_fence_after();
+                if (!(ok = wait(&bar_q[0], q_iter[0] & 1))) break;
+                ++q_iter[0];
+                tc_fence_after();
                 issue_s(0, kc % S);
-                if (n1 > 0) issue_s(1, kc % S);
-                if (n_max == 1) umma_commit_w(bar_q_free);
+                if (n0 == 1) umma_commit_w(&bar_q_free[0]);
+                if (n1 > 0) {
+                    if (!(ok = wait(&bar_q[1], q_iter[1] & 1))) break;
+                    ++q_iter[1];
+                    tc_fence_after();
+                    issue_s(1, kc % S);
+                    if (n1 == 1) umma_commit_w(&bar_q_free[1]);
+                }
+                umma_commit_w(&bar_kfree[kc % S]);
                 for (int j = 0; ok && j < n_max; ++j) {
                     const int s = (kc + j) % S;
                     const int s1 = (kc + j + 1) % S;
@@ -305,11 +327,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                                 k_ready = true;
                             }
                             issue_s(w, s1);
+                            if (j + 2 == nw) umma_commit_w(&bar_q_free[w]);  // last S_w of this unit issued
                         }
                     }
                     if (!ok) break;
-                    if (j + 2 == n_max) umma_commit_w(bar_q_free);  // last S of this unit issued
-                    umma_commit_w(&bar_empty[s]);
+                    if (j + 1 < n_max) umma_commit_w(&bar_kfree[s1]);
+                    umma_commit_w(&bar_vfree[s]);
                 }
                 kc += n_max;
             }
