@@ -6,6 +6,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <atomic>
 #include <mutex>
 
 #include "fa_internal.h"
@@ -14,6 +15,10 @@ namespace fa {
 namespace {
 
 __device__ int g_status;  // one per device; kernels record device-side conditions here
+// Forward unit schedulers: (ticket, finished-CTA count) pairs, used round-robin by
+// launches and reset to zero by the last CTA of each launch.
+constexpr unsigned kSchedSlots = 256;
+__device__ unsigned int g_fwd_sched[2 * kSchedSlots];
 
 constexpr int kMaxDevices = 64;
 
@@ -22,6 +27,8 @@ struct DeviceState {
     bool supported = false;
     int num_sms = 0;
     int* status_ptr = nullptr;
+    unsigned int* sched_ptr = nullptr;
+    std::atomic<unsigned> sched_next{0};
 };
 
 std::mutex g_mu;
@@ -49,6 +56,8 @@ int device_state(DeviceState** out) {
             void* ptr = nullptr;
             if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return FA_ERR_CUDA;
             st.status_ptr = static_cast<int*>(ptr);
+            if (cudaGetSymbolAddress(&ptr, g_fwd_sched) != cudaSuccess) return FA_ERR_CUDA;
+            st.sched_ptr = static_cast<unsigned int*>(ptr);
         }
         st.probed = true;
     }
@@ -167,6 +176,8 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     p.o = o;
     p.lse = lse;
     p.status = st->status_ptr;
+    // Launches in flight at the same time use different scheduler slots.
+    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
     p.B = B;
     p.H = H;
     p.Lq = Lq;

@@ -36,6 +36,7 @@ struct __align__(64) FwdParams {
     void* o;
     float* lse;
     int* status;
+    unsigned int* sched;  // [0]: next unit ticket, [1]: CTAs finished; both zero between launches
     int B, H, Lq, Lk;
     float scale;       // multiplies q.k
     float scale_log2;  // scale * log2(e)

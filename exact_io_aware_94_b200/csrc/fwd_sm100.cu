@@ -8,7 +8,10 @@
 //
 // B200 mapping.  A work unit is 256 query rows of one (b, h): two 128-row Q
 // tiles, one per softmax warpgroup.  The kernel is persistent (one CTA per SM)
-// and walks a static, balanced share of the units.  Each warpgroup's Q tile of
+// and claims units one at a time from the launch's ticket counter, in a fixed
+// heavy-first order, so the CTAs finish within a unit of one another.  The
+// producer warp claims each unit and hands it to the other roles through a
+// small ring in shared memory.  Each warpgroup's Q tile of
 // the next unit is loaded as soon as that warpgroup's last S MMA of the current
 // unit is done with the buffer, and a K slot is refilled once its S MMAs are
 // done (a V slot once its PV MMAs are), so loads, MMAs and the epilogue of
@@ -47,6 +50,7 @@ namespace fa {
 namespace {
 
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kUnitRing = 4;  // units published ahead by the producer
 
 
 
@@ -61,11 +65,12 @@ struct FwdLayout {
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
     // barriers: q[2], q_free[2], k[S], v[S], k_free[S], v_free[S], s[2], p[2][2 halves], o[2], o_free[2], drain
-    static constexpr int kNumBars = 4 + 4 * kStages + 10 + 1;
+    static constexpr int kNumBars = 4 + 4 * kStages + 10 + 1 + 2 * 4;  // + unit ring full/free
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // epilogue staging for the O tile stores: 4 KB per softmax warp (32 rows x 128 bytes,
     // 128-byte swizzle, so 1024-byte aligned)
-    static constexpr int kStageOff = (kMiscOff + 16 + 1023) / 1024 * 1024;
+    static constexpr int kRingOff = kMiscOff + 16;  // 4 unit indices
+    static constexpr int kStageOff = (kRingOff + 16 + 1023) / 1024 * 1024;
     static constexpr int kBytes = kStageOff + 8 * 4096 + 1024;  // + alignment slack
 };
 
@@ -126,19 +131,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint64_t* bar_o = bar_p + 4;
     uint64_t* bar_ofree = bar_o + 2;
     uint64_t* bar_drain = bar_ofree + 2;
+    // Unit ring: the producer claims units from the launch's ticket counter and
+    // publishes them here; the MMA warp and the 8 softmax warps read each entry.
+    uint64_t* bar_ufull = bar_drain + 1;
+    uint64_t* bar_ufree = bar_ufull + kUnitRing;
+    volatile int* s_unit = reinterpret_cast<volatile int*>(smem + Lay::kRingOff);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_units = p.B * p.H * ((p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
-    // Static boustrophedon assignment: in round r this CTA takes unit
-    // r*G + c (r even) or r*G + G-1-c (r odd).  Over the heavy-first order this
-    // balances the causal work across CTAs without any shared counter.
-    auto snake_unit = [&](int r) {
-        const int g = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-        return r * g + ((r & 1) ? g - 1 - c : c);
-    };
     const int off = p.Lk - p.Lq;
 
     // ---- setup
@@ -161,6 +164,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             mbar_init(&bar_ofree[w], 4 * 32);
         }
         mbar_init(bar_drain, 1);
+        for (int r = 0; r < kUnitRing; ++r) {
+            mbar_init(&bar_ufull[r], 1);
+            mbar_init(&bar_ufree[r], 1 + 8);  // MMA warp + 8 softmax warps
+        }
         *abort_flag = (atomicAdd(p.status, 0) == FA_ERR_TIMEOUT) ? 1 : 0;
         fence_barrier_init();
     }
@@ -194,7 +201,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             int nk = 0, nv = 0;        // K and V tiles whose loads were issued
             int q_iter[2] = {0, 0};    // Q tiles requested per warpgroup
             bool ok = true;
-            for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+            for (int it = 0; ok; ++it) {
+                // claim the next unit (heavy-first order) and publish it
+                const int rs = it % kUnitRing;
+                if (it >= kUnitRing && !(ok = wait(&bar_ufree[rs], ((it / kUnitRing) - 1) & 1))) break;
+                unsigned int ticket = 0;
+                if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+                const int u = static_cast<int>(min(__shfl_sync(0xffffffffu, ticket, 0), static_cast<unsigned>(n_units)));
+                if (lane == 0) {
+                    s_unit[rs] = u;
+                    mbar_arrive(&bar_ufull[rs]);
+                }
+                __syncwarp();
+                if (u >= n_units) break;
                 const Unit un = unit_of(p, u);
                 const int n_max = max(un.n_kv0, un.n_kv1);
                 // Q_w as soon as warpgroup w's S MMAs of its previous unit are done with the
@@ -274,7 +293,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             int tp[2] = {0, 0};        // P tiles consumed per warpgroup
             int units_w[2] = {0, 0};   // units whose O_w was handed to the epilogue
             bool ok = true;
-            for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+            for (int it = 0; ok; ++it) {
+                const int rs = it % kUnitRing;
+                if (!(ok = wait(&bar_ufull[rs], (it / kUnitRing) & 1))) break;
+                const int u = s_unit[rs];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_ufree[rs]);
+                if (u >= n_units) break;
                 const Unit un = unit_of(p, u);
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
@@ -353,7 +378,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         int ts = 0;      // S tiles consumed by this warpgroup
         int nunits = 0;  // units finished by this warpgroup
         bool ok = true;
-        for (int it = 0, u = snake_unit(0); ok && u < n_units; u = snake_unit(++it)) {
+        for (int it = 0; ok; ++it) {
+            const int rs = it % kUnitRing;
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar_ufull[rs], (it / kUnitRing) & 1, abort_flag, p.status));
+            if (!ok) break;
+            const int u = s_unit[rs];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_ufree[rs]);
+            if (u >= n_units) break;
             const Unit un = unit_of(p, u);
             const int n = (w == 0) ? un.n_kv0 : un.n_kv1;
             if (n == 0) continue;
@@ -529,6 +561,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem_base, 512);
+    }
+    // Every producer of this launch has stopped claiming units once it reaches here;
+    // the last CTA to finish returns the scheduler slot to zero for a later launch.
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.sched, 0u);
+            atomicExch(p.sched + 1, 0u);
+        }
     }
 }
 
