@@ -203,26 +203,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             constexpr uint32_t kIdescSS = idesc_bf16_f32(128, 128, 0, 0);
             constexpr uint32_t kIdescTS = idesc_bf16_f32(128, D, 0, 1);
             const uint32_t sKa = smem_u32(sK), sVa = smem_u32(sV), sQa = smem_u32(sQ), sGa = smem_u32(sG);
-            bool ok = wait(bar_kv, 0);
-            for (int t = 0; ok && t < nq; ++t) {
+            // S^T = K Q^T and dP^T = V dO^T for query tile t  (M = 128 keys, N = 128 queries, K = D)
+            auto issue_st = [&](int t) {
                 const int s = t % S;
-                if (!(ok = wait(&bar_qd[s], (t / S) & 1))) break;
-                tc_fence_after();
-                // S^T = K Q^T, dP^T = V dO^T   (M = 128 keys, N = 128 queries, K = D)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
                     umma_ss_w(tmem_base + kColS, smem_desc_sw128(sKa + koff, 16, 1024),
-                            smem_desc_sw128(sQa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                              smem_desc_sw128(sQa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
                 umma_commit_w(bar_s);
+            };
+            auto issue_dpt = [&](int t) {
+                const int s = t % S;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk >> 2) * T::kBoxBytes + (kk & 3) * 32;
                     umma_ss_w(tmem_base + kColDP, smem_desc_sw128(sVa + koff, 16, 1024),
-                            smem_desc_sw128(sGa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
+                              smem_desc_sw128(sGa + s * T::kTileBytes + koff, 16, 1024), kIdescSS, kk > 0);
                 }
                 umma_commit_w(bar_dp);
+            };
+            // Order per query tile t: dV(t), S^T(t+1), dK(t), dP^T(t+1).  S^T(t+1)
+            // overwrites the columns of P^T(t), so it follows dV(t), and dP^T(t+1)
+            // overwrites dS^T(t), so it follows dK(t); MMAs run in issue order.
+            // The next S^T is then computed while the elementwise warps form dS(t).
+            bool ok = wait(bar_kv, 0) && wait(&bar_qd[0], 0);
+            if (ok && nq > 0) {
+                tc_fence_after();
+                issue_st(0);
+                issue_dpt(0);
+            }
+            for (int t = 0; ok && t < nq; ++t) {
+                const int s = t % S;
+                const bool more = t + 1 < nq;
                 // dV += P^T dO   (A = P^T from TMEM: queries 0-63 at cols [0,32), 64-127 at [64,96))
                 if (!(ok = wait(bar_p, t & 1))) break;
                 tc_fence_after();
@@ -230,8 +244,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem_base + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
                     umma_ts_w(tmem_base + kColDV, a,
-                            smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
-                            (t > 0 || kk > 0) ? 1u : 0u);
+                              smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                              (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                if (more) {
+                    if (!(ok = wait(&bar_qd[(t + 1) % S], ((t + 1) / S) & 1))) break;
+                    tc_fence_after();
+                    issue_st(t + 1);
                 }
                 // dK += dS^T Q
                 if (!(ok = wait(bar_ds, t & 1))) break;
@@ -240,10 +259,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t a = tmem_base + kColDP + (kk >> 2) * 64 + (kk & 3) * 8;
                     umma_ts_w(tmem_base + kColDK, a,
-                            smem_desc_sw128(sQa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
-                            (t > 0 || kk > 0) ? 1u : 0u);
+                              smem_desc_sw128(sQa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                              (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit_w(&bar_empty[s]);
+                if (more) issue_dpt(t + 1);
             }
             if (ok) umma_commit_w(bar_acc);
             umma_commit_w(bar_drain);
