@@ -68,6 +68,45 @@ def decode_inputs(B: int, H: int, cap: int, d: int, seed: int, len_lo: int, len_
     return DecodeInputs(q, kc, vc, kv_lens)
 
 
+@dataclass
+class PagedDecodeInputs:
+    q: torch.Tensor            # [B, H, d] bf16
+    kpages: torch.Tensor       # [num_pages, Hkv, page_size, d] bf16
+    vpages: torch.Tensor       # [num_pages, Hkv, page_size, d] bf16
+    block_table: torch.Tensor  # int32 [B, max_blocks]
+    kv_lens: torch.Tensor      # int32 [B]
+
+
+def paged_decode_inputs(B: int, H: int, Hkv: int, page_size: int, max_blocks: int, d: int, seed: int,
+                        len_lo: int, len_hi: int, spare_pages: int = 0) -> PagedDecodeInputs:
+    """Paged decode workload.  Draw order: kv_lens ~ U{len_lo..len_hi}, then a random
+    permutation that assigns each used (sequence, block) a distinct page of the pool,
+    then q, then K pages and V pages (N(0,1), bf16).  Pages are [num_pages, Hkv,
+    page_size, d]; table slots past a sequence's last used block point at page 0, and
+    the pool has `spare_pages` pages that no sequence uses."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    kv_lens = torch.randint(len_lo, len_hi + 1, (B,), generator=gen, dtype=torch.int64).to(torch.int32)
+    used = [(int(n) + page_size - 1) // page_size for n in kv_lens]
+    num_pages = max(1, sum(used) + spare_pages)
+    perm = torch.randperm(num_pages, generator=gen)
+    table = torch.zeros((B, max_blocks), dtype=torch.int32)
+    at = 0
+    for b in range(B):
+        table[b, : used[b]] = perm[at:at + used[b]].to(torch.int32)
+        at += used[b]
+    q = _normal(gen, (B, H, d)).to(torch.bfloat16)
+    kp = torch.empty((num_pages, Hkv, page_size, d), dtype=torch.bfloat16)
+    vp = torch.empty((num_pages, Hkv, page_size, d), dtype=torch.bfloat16)
+    chunk = max(1, (1 << 24) // (Hkv * page_size * d))  # bounds the float32 temporaries
+    for p0 in range(0, num_pages, chunk):
+        p1 = min(num_pages, p0 + chunk)
+        kp[p0:p1] = _normal(gen, (p1 - p0, Hkv, page_size, d)).to(torch.bfloat16)
+    for p0 in range(0, num_pages, chunk):
+        p1 = min(num_pages, p0 + chunk)
+        vp[p0:p1] = _normal(gen, (p1 - p0, Hkv, page_size, d)).to(torch.bfloat16)
+    return PagedDecodeInputs(q, kp, vp, table, kv_lens)
+
+
 # The workloads the library is measured and checked on.  Shapes and value
 # distributions follow the pages' sizes: the 4,096-token example, a training
 # shape at 8,192, a 65,536-token context and a decode batch over a long cache.
@@ -77,4 +116,8 @@ WORKLOADS = {
     "train_L8192": dict(kind="fwdbwd", B=2, H=16, L=8192, d=128, causal=True, q_scale=1.0, seed=3),
     "long_L65536": dict(kind="fwd", B=1, H=8, L=65536, d=128, causal=True, q_scale=1.0, seed=4),
     "decode_cap32768": dict(kind="decode", B=64, H=32, cap=32768, d=128, len_lo=1024, len_hi=32768, seed=5),
+    # Paged cache with grouped heads: the same batch and lengths as the decode workload,
+    # 8 KV heads shared by groups of 4 query heads, 64-token pages in shuffled order.
+    "decode_paged_gqa": dict(kind="decode_paged", B=64, H=32, Hkv=8, page_size=64, max_blocks=512, d=128,
+                             len_lo=1024, len_hi=32768, seed=6),
 }

@@ -60,6 +60,9 @@ def _load():
                                         ctypes.c_double, c_int]
         lib.oracle_decode.restype = None
         lib.oracle_decode.argtypes = [vp, vp, vp, c_int, vp, dp, dp, i64, i64, i64, i64, ctypes.c_double]
+        lib.oracle_decode_paged.restype = c_int
+        lib.oracle_decode_paged.argtypes = [vp, vp, vp, c_int, vp, vp, dp, dp, i64, i64, i64, i64, i64, i64, i64,
+                                            ctypes.c_double]
         lib.oracle_merge.restype = None
         lib.oracle_merge.argtypes = [dp, dp, i64, i64, dp, dp]
         lib.oracle_num_threads.restype = c_int
@@ -186,6 +189,33 @@ def decode(q, kcache, vcache, kv_lens, scale: float):
     lse = np.empty((B, H), np.float64)
     _load().oracle_decode(pq, pk, pv, dt, lens.ctypes.data, o.ctypes.data, lse.ctypes.data, B, H, cap, d,
                           float(scale))
+    return o, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, kv_lens, scale: float):
+    """Single-query attention over a paged cache: q [B,H,d], pages [num_pages,Hkv,page_size,d],
+    block_table int32 [B, max_blocks], kv_lens int32 [B].  Query head h reads KV head h // (H // Hkv)."""
+    B, H, d = q.shape
+    num_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    kq, pq, cq = _as_input(q)
+    kk, pk, ck = _as_input(kpages)
+    kv, pv, cv = _as_input(vpages)
+    dt = _same_kind(cq, ck, cv)
+    bt = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    if bt.ndim != 2 or bt.shape[0] != B:
+        raise ValueError("block_table must have shape [B, max_blocks]")
+    lens = np.ascontiguousarray(np.asarray(kv_lens, dtype=np.int32))
+    if lens.shape != (B,):
+        raise ValueError("kv_lens must have shape [B]")
+    o = np.empty((B, H, d), np.float64)
+    lse = np.empty((B, H), np.float64)
+    rc = _load().oracle_decode_paged(pq, pk, pv, dt, bt.ctypes.data, lens.ctypes.data, o.ctypes.data,
+                                     lse.ctypes.data, B, H, Hkv, num_pages, page_size, bt.shape[1], d,
+                                     float(scale))
+    if rc == 1:
+        raise ValueError("a block-table entry used by a valid key is outside [0, num_pages)")
+    if rc == 2:
+        raise ValueError("H must be a multiple of Hkv")
     return o, lse
 
 

@@ -14,8 +14,10 @@
  *        mean bit-identical).
  *   [W]  "What Is FlashAttention? Why Long Context Got Cheap" -- "The problem it
  *        solves" (the textbook method builds the n x n score matrix, applies
- *        softmax, multiplies by V) and "What FlashAttention does instead"
- *        (running max and running sum per row).
+ *        softmax, multiplies by V), "What FlashAttention does instead"
+ *        (running max and running sum per row), "What it changes for you"
+ *        (the key/value cache kept in HBM during generation) and "The general
+ *        lesson" (paged attention named among the data-movement techniques).
  *   [L]  "How Flash Attention Improves Transformer Memory Efficiency Compared
  *        to Standard Attention" -- "The Three Running Statistics" (the m, l and
  *        unnormalised-output update rules and the final division), "Backward
@@ -315,6 +317,76 @@ void oracle_decode(const void* q, const void* kcache, const void* vcache, int dt
         }
         free(t);
     }
+}
+
+/*
+ * Single-query attention over a paged cache.  [W] "What it changes for you":
+ * during generation the keys and values of every processed token are kept in
+ * a cache in HBM that grows with each token; [W] "The general lesson" names
+ * paged attention among the ways of moving less data.  Here a sequence's cache
+ * is a list of fixed-size pages: logical key j of sequence b is row
+ * j % page_size of page block_table[b * max_blocks + j / page_size].  Pages are
+ * laid out [num_pages, Hkv, page_size, d].  Query heads share key/value heads
+ * in equal groups: query head h reads KV head h / (H / Hkv).
+ * The result is plain attention (as oracle_decode) over keys [0, kv_len_b),
+ * kv_len clamped to [0, max_blocks * page_size].
+ * Returns 0, or 1 if a page index that a valid key would use is outside
+ * [0, num_pages) (nothing is read then), or 2 if H is not a multiple of Hkv.
+ */
+int oracle_decode_paged(const void* q, const void* kpages, const void* vpages, int dtype,
+                        const int32_t* block_table, const int32_t* kv_lens, double* o,
+                        double* lse, int64_t B, int64_t H, int64_t Hkv, int64_t num_pages,
+                        int64_t page_size, int64_t max_blocks, int64_t d, double scale) {
+    if (Hkv <= 0 || H % Hkv != 0 || page_size <= 0) return 2;
+    const int64_t group = H / Hkv;
+    const int64_t cap = max_blocks * page_size;
+    for (int64_t b = 0; b < B; ++b) {
+        int64_t n = kv_lens[b];
+        if (n < 0) n = 0;
+        if (n > cap) n = cap;
+        for (int64_t blk = 0; blk * page_size < n; ++blk) {
+            const int32_t pg = block_table[b * max_blocks + blk];
+            if (pg < 0 || pg >= num_pages) return 1;
+        }
+    }
+    const int64_t heads = B * H;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(cap > 0 ? cap : 1));
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < heads; ++bh) {
+            const int64_t b = bh / H, h = bh % H, g = h / group;
+            int64_t n = kv_lens[b];
+            if (n < 0) n = 0;
+            if (n > cap) n = cap;
+            double* orow = o + bh * d;
+            for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+            if (n == 0) {
+                lse[bh] = -INFINITY;
+                continue;
+            }
+            double M = -INFINITY;
+            for (int64_t j = 0; j < n; ++j) {
+                const int64_t pg = block_table[b * max_blocks + j / page_size];
+                const int64_t row = ((pg * Hkv + g) * page_size + j % page_size) * d;
+                double sdot = 0.0;
+                for (int64_t c = 0; c < d; ++c) sdot += elem(q, bh * d + c, dtype) * elem(kpages, row + c, dtype);
+                t[j] = scale * sdot;
+                if (t[j] > M) M = t[j];
+            }
+            double Z = 0.0;
+            for (int64_t j = 0; j < n; ++j) Z += exp(t[j] - M);
+            for (int64_t j = 0; j < n; ++j) {
+                const int64_t pg = block_table[b * max_blocks + j / page_size];
+                const int64_t row = ((pg * Hkv + g) * page_size + j % page_size) * d;
+                const double pj = exp(t[j] - M) / Z;
+                for (int64_t c = 0; c < d; ++c) orow[c] += pj * elem(vpages, row + c, dtype);
+            }
+            lse[bh] = M + log(Z);
+        }
+        free(t);
+    }
+    return 0;
 }
 
 /*

@@ -268,3 +268,86 @@ def test_backward_single_key_closed_form():
     np.testing.assert_allclose(dq, 0.0, atol=1e-15)
     np.testing.assert_allclose(dk, 0.0, atol=1e-15)
     np.testing.assert_allclose(dv[0, 0, 0], g[0, 0].sum(axis=0), atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- paged, grouped-head decode
+def _paged_from_cache(kc, vc, page_size, order):
+    """Cut contiguous caches [B, Hkv, cap, d] into pages [B*nblk, Hkv, page_size, d]; page
+    order[b*nblk + blk] holds block blk of sequence b.  Returns (kpages, vpages, table)."""
+    B, Hkv, cap, d = kc.shape
+    nblk = cap // page_size
+    kp = torch.empty((B * nblk, Hkv, page_size, d), dtype=kc.dtype)
+    vp = torch.empty_like(kp)
+    table = np.zeros((B, nblk), np.int32)
+    for b in range(B):
+        for blk in range(nblk):
+            pg = int(order[b * nblk + blk])
+            kp[pg] = kc[b, :, blk * page_size:(blk + 1) * page_size]
+            vp[pg] = vc[b, :, blk * page_size:(blk + 1) * page_size]
+            table[b, blk] = pg
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("permute", [False, True])
+def test_paged_decode_equals_contiguous_decode(permute):
+    """With one KV head per query head, gathering through the block table must give
+    exactly the contiguous-cache decode, whatever order the pages are stored in."""
+    g = torch.Generator("cpu").manual_seed(11)
+    B, H, cap, d, ps = 3, 2, 48, 8, 16
+    kc = torch.randn(B, H, cap, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, H, cap, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    lens = np.array([1, 31, 48], np.int32)  # single key, mid-page end, full capacity
+    order = np.random.default_rng(3).permutation(B * cap // ps) if permute else np.arange(B * cap // ps)
+    kp, vp, table = _paged_from_cache(kc, vc, ps, order)
+    o_p, l_p = oracle.decode_paged(q, kp, vp, table, lens, 0.3)
+    o_c, l_c = oracle.decode(q, kc, vc, lens, 0.3)
+    assert np.max(np.abs(o_p - o_c)) <= 1e-12
+    assert np.max(np.abs(l_p - l_c)) <= 1e-12
+
+
+def test_paged_decode_grouped_heads_equal_replicated_cache():
+    """Query head h reads KV head h // (H // Hkv): equal to a contiguous decode whose
+    cache repeats each KV head for its group of query heads."""
+    g = torch.Generator("cpu").manual_seed(12)
+    B, H, Hkv, cap, d, ps = 2, 8, 2, 32, 8, 8
+    kc = torch.randn(B, Hkv, cap, d, generator=g).to(torch.bfloat16)
+    vc = torch.randn(B, Hkv, cap, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    lens = np.array([29, 17], np.int32)
+    kp, vp, table = _paged_from_cache(kc, vc, ps, np.random.default_rng(5).permutation(B * cap // ps))
+    o_p, l_p = oracle.decode_paged(q, kp, vp, table, lens, 0.25)
+    group = H // Hkv
+    kr = kc.repeat_interleave(group, dim=1)  # [B, H, cap, d]: head h holds KV head h // group
+    vr = vc.repeat_interleave(group, dim=1)
+    o_c, l_c = oracle.decode(q, kr, vr, lens, 0.25)
+    assert np.max(np.abs(o_p - o_c)) <= 1e-12
+    assert np.max(np.abs(l_p - l_c)) <= 1e-12
+    # heads of one group see the same keys but different queries: results differ across the group
+    assert np.max(np.abs(o_p[:, 0] - o_p[:, 1])) > 1e-3
+
+
+def test_paged_decode_unused_slots_and_errors():
+    g = torch.Generator("cpu").manual_seed(13)
+    B, H, Hkv, d, ps, nblk = 2, 4, 2, 4, 4, 3
+    kp = torch.randn(5, Hkv, ps, d, generator=g).to(torch.bfloat16)
+    vp = torch.randn(5, Hkv, ps, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(B, H, d, generator=g).to(torch.bfloat16)
+    table = np.array([[2, 0, 4], [1, 3, 0]], np.int32)
+    lens = np.array([6, 0], np.int32)  # sequence 0 uses blocks 0-1; sequence 1 is empty
+    o, l = oracle.decode_paged(q, kp, vp, table, lens, 0.5)
+    # entries past the last used block are never read
+    t2 = table.copy()
+    t2[0, 2] = 10 ** 6
+    t2[1, :] = -7
+    o2, l2 = oracle.decode_paged(q, kp, vp, t2, lens, 0.5)
+    assert np.array_equal(o, o2) and np.array_equal(l, l2)
+    # an empty sequence gives O = 0 and LSE = -inf
+    assert np.all(o[1] == 0.0) and np.all(np.isneginf(l[1]))
+    # a used entry outside [0, num_pages) is an error, and so is H not a multiple of Hkv
+    t3 = table.copy()
+    t3[0, 1] = 5
+    with pytest.raises(ValueError):
+        oracle.decode_paged(q, kp, vp, t3, lens, 0.5)
+    with pytest.raises(ValueError):
+        oracle.decode_paged(torch.randn(B, 3, d).to(torch.bfloat16), kp, vp, table, lens, 0.5)
