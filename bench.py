@@ -434,6 +434,45 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "l2": "caches 2 x 16 GiB, far larger than L2",
                                "traffic": recorded_traffic("fa_decode", "decode_cap32768", ["decode_sm100.cu"])}
     del kc, vc
+
+    # paged cache with grouped heads: same batch and lengths, 8 KV heads for 32 query heads
+    w = WORKLOADS["decode_paged_gqa"]
+    B, H, Hkv, ps, nblk, d = w["B"], w["H"], w["Hkv"], w["page_size"], w["max_blocks"], w["d"]
+    cg = torch.Generator("cpu").manual_seed(w["seed"])
+    lens = torch.randint(w["len_lo"], w["len_hi"] + 1, (B,), generator=cg).to(torch.int32)
+    used = [(int(n) + ps - 1) // ps for n in lens]
+    num_pages = sum(used)
+    perm = torch.randperm(num_pages, generator=cg).to(torch.int32)
+    table = torch.zeros(B, nblk, dtype=torch.int32)
+    at = 0
+    for b in range(B):
+        table[b, : used[b]] = perm[at:at + used[b]]
+        at += used[b]
+    kp = torch.randn(num_pages, Hkv, ps, d, generator=gen, device=device).to(torch.bfloat16)
+    vp = torch.randn(num_pages, Hkv, ps, d, generator=gen, device=device).to(torch.bfloat16)
+    qp = torch.randn(B, H, d, generator=gen, device=device).to(torch.bfloat16)
+    table_d, lens_p = table.to(device), lens.to(device)
+    op = torch.empty(B, H, d, dtype=torch.float32, device=device)
+    lp = torch.empty(B, H, dtype=torch.float32, device=device)
+    wsp = fa.workspace(fa.fa_decode_paged_workspace_size(B, H, nblk, ps, d), device)
+
+    def dec_paged():
+        rc = fa.fa_decode_paged(qp, kp, vp, table_d, lens_p, op, lp, B, H, Hkv, num_pages, ps, nblk, d, scale,
+                                fa.FA_DT_F32, wsp, wsp.numel(), stream)
+        assert rc == fa.FA_OK
+
+    nbytes = int(lens.sum()) * Hkv * d * 2 * 2
+    t_p = time_steps(dec_paged, steps, warm, stream, dist, device) / steps
+    legs["decode_paged_gqa"] = {"ms": round(t_p * 1e3, 4), "GB/s": round(nbytes / t_p / 1e9, 1),
+                                "kv_bytes": nbytes,
+                                "frac_of_peak": round(nbytes / t_p / 1e9 / peaks["hbm_gbs"], 4),
+                                "frac_of_nominal_8000": round(nbytes / t_p / 1e9 / NOMINAL_HBM_GBS, 4),
+                                "launches": 3,
+                                "kernels": "fa_decode_plan + fa_decode_paged_split + fa_decode_combine",
+                                "config": "B64 H32 Hkv8 (groups of 4) d128, 64-token pages in shuffled order, "
+                                          "lengths U[1024, 32768]",
+                                "l2": "pages 2 x %.1f GiB, far larger than L2" % (kp.numel() * 2 / 2 ** 30)}
+    del kp, vp
     status = fa.fa_check_status(stream)
     if status != fa.FA_OK:
         raise fa.FAError(status, "device status after the legs")

@@ -36,6 +36,7 @@ FA_ERR_TIMEOUT = 5
 FA_ERR_DEVICE = 6
 FA_ERR_KV_LEN = 7
 FA_ERR_TOO_LARGE = 8
+FA_ERR_PAGE = 9
 FA_NOALLOC_MAX_ROWS = 1 << 20
 FA_DT_BF16 = 0
 FA_DT_F32 = 1
@@ -73,6 +74,10 @@ def load_library():
     lib.fa_decode_workspace_size.argtypes = [i, i, i, i]
     lib.fa_decode.restype = i
     lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_decode_paged_workspace_size.restype = sz
+    lib.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_decode_paged.restype = i
+    lib.fa_decode_paged.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_check_status.restype = i
     lib.fa_check_status.argtypes = [vp]
     lib.fa_status_string.restype = ctypes.c_char_p
@@ -135,6 +140,18 @@ def fa_decode(q, kcache, vcache, kv_lens, o, lse, B, H, cap, d, scale, o_dtype, 
     return load_library().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(o), _ptr(lse), B,
                                     H, cap, d, float(scale), int(o_dtype), _ptr(workspace), int(workspace_bytes),
                                     _stream(stream))
+
+
+def fa_decode_paged_workspace_size(B, H, max_blocks, page_size, d) -> int:
+    return int(load_library().fa_decode_paged_workspace_size(B, H, max_blocks, page_size, d))
+
+
+def fa_decode_paged(q, kpages, vpages, block_table, kv_lens, o, lse, B, H, Hkv, num_pages, page_size, max_blocks, d,
+                    scale, o_dtype, workspace, workspace_bytes, stream=None) -> int:
+    return load_library().fa_decode_paged(_ptr(q), _ptr(kpages), _ptr(vpages), _ptr(block_table), _ptr(kv_lens),
+                                          _ptr(o), _ptr(lse), B, H, Hkv, num_pages, page_size, max_blocks, d,
+                                          float(scale), int(o_dtype), _ptr(workspace), int(workspace_bytes),
+                                          _stream(stream))
 
 
 def fa_check_status(stream=None) -> int:
@@ -215,4 +232,27 @@ def decode(q, kcache, vcache, kv_lens, scale=None, out_dtype=torch.float32, ws=N
     rc = fa_decode(q, kcache, vcache, kv_lens, o, lse, B, H, cap, d, scale, _DT[out_dtype], ws,
                    ws.numel() * ws.element_size(), stream)
     _check(rc, "fa_decode")
+    return o, lse
+
+
+def decode_paged(q, kpages, vpages, block_table, kv_lens, scale=None, out_dtype=torch.float32, ws=None, stream=None):
+    """o [B,H,d] and lse [B,H] for q [B,H,d], pages [num_pages,Hkv,page_size,d] (bf16),
+    block_table int32 [B,max_blocks] and kv_lens int32 [B] (device)."""
+    for t, n in ((q, "q"), (kpages, "kpages"), (vpages, "vpages")):
+        _need(t, n)
+    _need(block_table, "block_table", torch.int32)
+    _need(kv_lens, "kv_lens", torch.int32)
+    B, H, d = q.shape
+    num_pages, Hkv, page_size = kpages.shape[0], kpages.shape[1], kpages.shape[2]
+    max_blocks = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    nbytes = fa_decode_paged_workspace_size(B, H, max_blocks, page_size, d)
+    if ws is None:
+        ws = workspace(nbytes, q.device)
+    o = torch.empty((B, H, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    rc = fa_decode_paged(q, kpages, vpages, block_table, kv_lens, o, lse, B, H, Hkv, num_pages, page_size, max_blocks,
+                         d, scale, _DT[out_dtype], ws, ws.numel() * ws.element_size(), stream)
+    _check(rc, "fa_decode_paged")
     return o, lse

@@ -146,6 +146,8 @@ const char* fa_status_string(int status) {
         case FA_ERR_KV_LEN: return "FA_ERR_KV_LEN: a decode cache length was outside [0, cap]";
         case FA_ERR_TOO_LARGE:
             return "FA_ERR_TOO_LARGE: B*H*Lq exceeds FA_NOALLOC_MAX_ROWS, the fixed scratch of fa_backward_noalloc";
+        case FA_ERR_PAGE:
+            return "FA_ERR_PAGE: a block-table entry used by a valid key was outside [0, num_pages) (read as page 0)";
         default: return "unknown fa_status";
     }
 }
@@ -284,6 +286,64 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o, cons
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
     cudaError_t e = launch_bwd(p, d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_decode_paged_workspace_size(int B, int H, int max_blocks, int page_size, int d) {
+    if (B <= 0 || H <= 0 || max_blocks <= 0 || page_size <= 0 || (d != 64 && d != 128)) return 0;
+    const long long cap = static_cast<long long>(max_blocks) * page_size;
+    if (cap > 0x7FFFFFFFLL) return 0;
+    return decode_workspace_bytes(B, H, static_cast<int>(cap), d);
+}
+
+int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                    const int* kv_lens, void* o, float* lse, int B, int H, int Hkv, int num_pages, int page_size,
+                    int max_blocks, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+    if (!q || !kpages || !vpages || !block_table || !kv_lens || !o || !lse) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || num_pages <= 0 || max_blocks <= 0) return FA_ERR_INVALID_ARG;
+    if (page_size <= 0 || page_size > 65536 || (page_size & (page_size - 1)) != 0) return FA_ERR_INVALID_ARG;
+    const long long cap = static_cast<long long>(max_blocks) * page_size;
+    if (cap > 0x7FFFFFFFLL || static_cast<long long>(B) * H > (1LL << 30) ||
+        static_cast<long long>(B) * max_blocks > 0x7FFFFFFFLL)
+        return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(kpages, 16) || !aligned(vpages, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(block_table, 4) || !aligned(kv_lens, 4))
+        return FA_ERR_INVALID_ARG;
+    const size_t need = decode_workspace_bytes(B, H, static_cast<int>(cap), d);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return FA_ERR_WORKSPACE;
+    const long long max_splits = (cap + kDecodeSplit - 1) / kDecodeSplit;
+    if (static_cast<long long>(B) * H * max_splits > 0x7FFFFFFFLL) return FA_ERR_INVALID_ARG;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    DecodeParams p{};
+    p.q = q;
+    p.k = kpages;
+    p.v = vpages;
+    p.kv_lens = kv_lens;
+    p.o = o;
+    p.lse = lse;
+    p.status = st->status_ptr;
+    p.B = B;
+    p.H = H;
+    p.cap = static_cast<int>(cap);
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.o_dtype = o_dtype;
+    p.block_table = block_table;
+    p.Hkv = Hkv;
+    p.num_pages = num_pages;
+    int shift = 0;
+    while ((1 << shift) < page_size) ++shift;
+    p.page_shift = shift;
+    p.max_blocks = max_blocks;
+    decode_carve_workspace(p, workspace, B, H, static_cast<int>(cap), d);
+    cudaError_t e = launch_decode_paged(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -15,6 +15,14 @@
 //                      prefix-sums the chunk counts per sequence.
 //   fa_decode_split    persistent CTAs over all (b, h, chunk) items.
 //   fa_decode_combine  one CTA per (b, h): log-sum-exp merge of its chunks.
+//
+// Paged cache with grouped heads (fa_decode_paged): the same split and combine,
+// with keys reached through a per-sequence block table of fixed-size pages and
+// H / Hkv query heads sharing each key/value head ("What Is FlashAttention?",
+// "The general lesson" names paged attention among the ways of moving less
+// data).  A work item covers a group of query heads of one KV head, so every K
+// and V row it loads serves the whole group.
+//   fa_decode_paged_split  persistent CTAs over (b, kv head, head group, chunk).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -67,6 +75,14 @@ __global__ void __launch_bounds__(kPlanThreads) fa_decode_plan(DecodeParams p) {
         }
         p.lens[b] = n;
         local += (n + kDecodeSplit - 1) / kDecodeSplit;
+        if (p.block_table) {
+            // every page a valid key will read must exist; the split kernel clamps bad ones
+            const int nblk = (n + (1 << p.page_shift) - 1) >> p.page_shift;
+            for (int blk = 0; blk < nblk; ++blk) {
+                const int pg = p.block_table[static_cast<size_t>(b) * p.max_blocks + blk];
+                if (pg < 0 || pg >= p.num_pages) atomicCAS(p.status, 0, FA_ERR_PAGE);
+            }
+        }
     }
     part[t] = local;
     __syncthreads();
@@ -209,6 +225,187 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) fa_decode_split(DecodeParam
     }
 }
 
+// Paged cache, GG query heads per work item sharing one KV head.  Same lane
+// layout as fa_decode_split: D/8 lanes hold one key row; each lane keeps the
+// running statistics of all GG heads for its slice of keys.
+template <int D, int GG, int UNROLL, int MINB>
+__global__ void __launch_bounds__(kDecodeThreads, MINB) fa_decode_paged_split(DecodeParams p) {
+    constexpr int kLanesPerKey = D / 8;
+    constexpr int kGroupsPerWarp = 32 / kLanesPerKey;
+    constexpr int kGroups = (kDecodeThreads / 32) * kGroupsPerWarp;
+    constexpr int kStep = kGroups * UNROLL;
+
+    __shared__ float red_m[GG][kGroups];
+    __shared__ float red_l[GG][kGroups];
+    __shared__ float red_acc[GG][kGroups][D];
+    __shared__ int s_item[4];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;
+    const int e0 = (lane % kLanesPerKey) * 8;
+    const float sl2 = p.scale_log2;
+    const int group = p.H / p.Hkv;      // query heads per KV head
+    const int n_hg = group / GG;        // head groups per KV head
+    const int per_chunk = p.Hkv * n_hg;  // items per chunk of a sequence
+    const int total = p.cum[p.B] * per_chunk;
+    const int ps_mask = (1 << p.page_shift) - 1;
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        if (threadIdx.x == 0) {
+            // item -> (b, kv head, chunk, head group), ordered by b, then kv head, then
+            // chunk, then head group: the head groups of one chunk run side by side, so
+            // all but the first find that chunk's K and V rows in L2.
+            int lo = 0, hi = p.B;
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (p.cum[mid] * per_chunk <= item) lo = mid; else hi = mid;
+            }
+            const int nb = p.cum[lo + 1] - p.cum[lo];
+            const int local = item - p.cum[lo] * per_chunk;
+            const int rem = local % (nb * n_hg);
+            s_item[0] = lo;
+            s_item[1] = local / (nb * n_hg);  // kv head
+            s_item[2] = rem % n_hg;           // head group
+            s_item[3] = rem / n_hg;           // chunk
+        }
+        __syncthreads();
+        const int b = s_item[0], hkv = s_item[1], hg = s_item[2], chunk = s_item[3];
+        const int h0 = hkv * group + hg * GG;  // first query head of this item
+        const int len = p.lens[b];
+        const int start = chunk * kDecodeSplit;
+        const int end = min(start + kDecodeSplit, len);
+        const int* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+        const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k) + e0;
+        const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.v) + e0;
+
+        // q as packed pairs (x = element 2i, y = element 2i+1) for FFMA2
+        float2 q2[GG][4];
+#pragma unroll
+        for (int gg = 0; gg < GG; ++gg) {
+            float qf[8];
+            unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                    (static_cast<size_t>(b) * p.H + h0 + gg) * D + e0),
+                    qf);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) q2[gg][i] = make_float2(qf[2 * i], qf[2 * i + 1]);
+        }
+        // Running statistics per head against a reference max m (deferred rescale:
+        // O = acc / l holds for any common reference, so acc and l are rescaled only
+        // when a head's max has grown by more than 2^8 in exp2 units).
+        float m[GG], l[GG];
+        float2 acc2[GG][4];
+#pragma unroll
+        for (int gg = 0; gg < GG; ++gg) {
+            m[gg] = -INFINITY;
+            l[gg] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc2[gg][i] = make_float2(0.0f, 0.0f);
+        }
+
+        for (int base = start; base < end; base += kStep) {
+            uint4 kr[UNROLL], vr[UNROLL];
+            bool valid[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int key = base + u * kGroups + g;
+                valid[u] = key < end;
+                int pg = valid[u] ? table[key >> p.page_shift] : 0;
+                pg = (static_cast<unsigned>(pg) < static_cast<unsigned>(p.num_pages)) ? pg : 0;  // flagged by the plan
+                const size_t row = (static_cast<size_t>(pg) * p.Hkv + hkv) * (ps_mask + 1) + (key & ps_mask);
+                kr[u] = valid[u] ? ld_stream_u4(kbase + row * D) : make_uint4(0, 0, 0, 0);
+                vr[u] = valid[u] ? ld_stream_u4(vbase + row * D) : make_uint4(0, 0, 0, 0);
+            }
+            float s[UNROLL][GG];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const float2 k2[4] = {make_float2(__uint_as_float(kr[u].x << 16), __uint_as_float(kr[u].x & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(kr[u].y << 16), __uint_as_float(kr[u].y & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(kr[u].z << 16), __uint_as_float(kr[u].z & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(kr[u].w << 16), __uint_as_float(kr[u].w & 0xFFFF0000u))};
+#pragma unroll
+                for (int gg = 0; gg < GG; ++gg) {
+                    float2 d2 = __fmul2_rn(q2[gg][0], k2[0]);
+#pragma unroll
+                    for (int i = 1; i < 4; ++i) d2 = __ffma2_rn(q2[gg][i], k2[i], d2);
+                    float dot = d2.x + d2.y;
+#pragma unroll
+                    for (int o = kLanesPerKey / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                    s[u][gg] = valid[u] ? dot : -INFINITY;
+                }
+            }
+            bool grow = false;
+            float mb[GG];
+#pragma unroll
+            for (int gg = 0; gg < GG; ++gg) {
+                mb[gg] = s[0][gg];
+#pragma unroll
+                for (int u = 1; u < UNROLL; ++u) mb[gg] = fmaxf(mb[gg], s[u][gg]);
+                grow |= (m[gg] == -INFINITY) ? (mb[gg] != -INFINITY) : ((mb[gg] - m[gg]) * sl2 > 8.0f);
+            }
+            if (__any_sync(0xffffffffu, grow)) {  // warp-uniform, rare after the first keys
+#pragma unroll
+                for (int gg = 0; gg < GG; ++gg) {
+                    const float m_new = fmaxf(m[gg], mb[gg]);
+                    const float alpha = (m[gg] == -INFINITY) ? 0.0f : ex2f_approx((m[gg] - m_new) * sl2);
+                    l[gg] *= alpha;
+                    const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc2[gg][i] = __fmul2_rn(acc2[gg][i], a2);
+                    m[gg] = m_new;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const float2 v2[4] = {make_float2(__uint_as_float(vr[u].x << 16), __uint_as_float(vr[u].x & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(vr[u].y << 16), __uint_as_float(vr[u].y & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(vr[u].z << 16), __uint_as_float(vr[u].z & 0xFFFF0000u)),
+                                      make_float2(__uint_as_float(vr[u].w << 16), __uint_as_float(vr[u].w & 0xFFFF0000u))};
+#pragma unroll
+                for (int gg = 0; gg < GG; ++gg) {
+                    // m = -inf only while no valid key was seen: then every p is 0
+                    const float mbias = (m[gg] == -INFINITY) ? 0.0f : m[gg] * sl2;
+                    const float pu = ex2f_approx(fmaf(s[u][gg], sl2, -mbias));  // 0 for invalid keys
+                    l[gg] += pu;
+                    const float2 p2 = make_float2(pu, pu);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc2[gg][i] = __ffma2_rn(p2, v2[i], acc2[gg][i]);
+                }
+            }
+        }
+
+        // merge the key groups of this CTA, per head
+#pragma unroll
+        for (int gg = 0; gg < GG; ++gg) {
+            if (lane % kLanesPerKey == 0) {
+                red_m[gg][g] = m[gg];
+                red_l[gg][g] = l[gg];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                red_acc[gg][g][e0 + 2 * i] = acc2[gg][i].x;
+                red_acc[gg][g][e0 + 2 * i + 1] = acc2[gg][i].y;
+            }
+        }
+        __syncthreads();
+        for (int t = threadIdx.x; t < GG * D; t += kDecodeThreads) {
+            const int gg = t / D, c = t % D;
+            float M = -INFINITY;
+            for (int i = 0; i < kGroups; ++i) M = fmaxf(M, red_m[gg][i]);
+            float L = 0.0f, O = 0.0f;
+            for (int i = 0; i < kGroups; ++i) {
+                if (red_m[gg][i] == -INFINITY) continue;
+                const float w = ex2f_approx((red_m[gg][i] - M) * sl2);
+                L = fmaf(w, red_l[gg][i], L);
+                O = fmaf(w, red_acc[gg][i][c], O);
+            }
+            const size_t slot = (static_cast<size_t>(b) * p.H + h0 + gg) * p.max_splits + chunk;
+            p.part_o[slot * D + c] = O / L;
+            if (c == 0) p.part_lse[slot] = M * p.scale + logf(L);
+        }
+        __syncthreads();
+    }
+}
+
 template <int D>
 __global__ void __launch_bounds__(D) fa_decode_combine(DecodeParams p) {
     const int bh = blockIdx.x;
@@ -238,7 +435,47 @@ __global__ void __launch_bounds__(D) fa_decode_combine(DecodeParams p) {
     if (c == 0) p.lse[bh] = M + logf(L);
 }
 
+template <int D, int GG, int UNROLL, int MINB>
+cudaError_t launch_paged_split(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+    const int n_hg = (p.H / p.Hkv) / GG;
+    const long long upper = static_cast<long long>(p.B) * p.Hkv * n_hg * p.max_splits;
+    const int grid = static_cast<int>(std::min<long long>(upper, static_cast<long long>(num_sms) * MINB));
+    fa_decode_paged_split<D, GG, UNROLL, MINB><<<grid, kDecodeThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+// Head-group width and, for groups of 4, unroll depth and CTAs per SM.  Groups of
+// 4 measured fastest (smaller groups re-read K/V through L2); 3 keys in flight per
+// lane group at 2 CTAs per SM beat 2 keys, and 4 keys at 1 CTA per SM.
+#ifndef FA_PAGED_GG
+#define FA_PAGED_GG 4
+#endif
+#ifndef FA_PG4_U
+#define FA_PG4_U 3
+#endif
+#ifndef FA_PG4_M
+#define FA_PG4_M 2
+#endif
+template <int D>
+cudaError_t launch_paged_d(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+    const int group = p.H / p.Hkv;
+    cudaError_t e;
+    if (FA_PAGED_GG >= 4 && group % 4 == 0) e = launch_paged_split<D, 4, FA_PG4_U, FA_PG4_M>(p, num_sms, stream);
+    else if (FA_PAGED_GG >= 2 && group % 2 == 0) e = launch_paged_split<D, 2, 4, 2>(p, num_sms, stream);
+    else e = launch_paged_split<D, 1, 4, 3>(p, num_sms, stream);
+    if (e != cudaSuccess) return e;
+    fa_decode_combine<D><<<p.B * p.H, D, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaStream_t stream) {
+    fa_decode_plan<<<1, kPlanThreads, 0, stream>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return d == 128 ? launch_paged_d<128>(p, num_sms, stream) : launch_paged_d<64>(p, num_sms, stream);
+}
 
 size_t decode_workspace_bytes(int B, int H, int cap, int d) {
     const size_t max_splits = (static_cast<size_t>(cap) + kDecodeSplit - 1) / kDecodeSplit;

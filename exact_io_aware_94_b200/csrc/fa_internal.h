@@ -91,11 +91,15 @@ struct DecodeParams {
     int B, H, cap, max_splits;
     float scale, scale_log2;
     int o_dtype;
+    // paged cache (fa_decode_paged); block_table is null for the contiguous cache
+    const int* block_table;  // [B, max_blocks] page indices
+    int Hkv, num_pages, page_shift, max_blocks;  // page_size = 1 << page_shift
 };
 
 size_t decode_workspace_bytes(int B, int H, int cap, int d);
 void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, int d);
 cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
+cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 
 int fwd_smem_bytes(int d);
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);

@@ -58,7 +58,8 @@ typedef enum {
     FA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
     FA_ERR_DEVICE = 6,      /* current device is not compute capability 10.0 */
     FA_ERR_KV_LEN = 7,      /* device: a decode cache length was outside [0, cap] (clamped) */
-    FA_ERR_TOO_LARGE = 8    /* problem larger than the fixed scratch of fa_backward_noalloc */
+    FA_ERR_TOO_LARGE = 8,   /* problem larger than the fixed scratch of fa_backward_noalloc */
+    FA_ERR_PAGE = 9         /* device: a block-table entry used by a valid key was outside [0, num_pages) */
 } fa_status;
 
 enum { FA_DT_BF16 = 0, FA_DT_F32 = 1 };
@@ -141,6 +142,44 @@ size_t fa_decode_workspace_size(int B, int H, int cap, int d);
 int fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens, void* o, float* lse,
               int B, int H, int cap, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
               void* stream);
+
+/*
+ * Workspace bytes fa_decode_paged needs: the same split-KV partials as
+ * fa_decode for B*H query heads and a logical capacity of
+ * max_blocks * page_size keys.
+ */
+size_t fa_decode_paged_workspace_size(int B, int H, int max_blocks, int page_size, int d);
+
+/*
+ * Single-query decode over a paged KV cache with grouped key/value heads.
+ * Source: "What Is FlashAttention?", "What it changes for you" (the key/value
+ * cache of a generation lives in HBM and grows with every token) and "The
+ * general lesson" (paged attention named among the data-movement techniques);
+ * the attention itself is the same as fa_decode.
+ *   q           [B, H, d] bf16.
+ *   kpages,
+ *   vpages      [num_pages, Hkv, page_size, d] bf16: page p holds page_size
+ *               consecutive token positions of one sequence, for every KV head.
+ *   block_table int32 [B, max_blocks] on the device: logical key j of sequence
+ *               b is row j % page_size of page block_table[b][j / page_size].
+ *   kv_lens     int32 [B] on the device, valid keys per sequence.
+ *   o, lse      [B, H, d] (o_dtype) and [B, H] fp32.
+ * Query head h reads KV head h / (H / Hkv).  H must be a multiple of Hkv and
+ * page_size a power of two (1 .. 65536); d is 64 or 128.  q, kpages, vpages and
+ * o must be 16-byte aligned, the workspace 256-byte aligned (any torch
+ * allocation is).  Lengths outside [0, max_blocks *
+ * page_size] are clamped and flagged FA_ERR_KV_LEN; a table entry that a valid
+ * key uses and that lies outside [0, num_pages) is flagged FA_ERR_PAGE in the
+ * status word and read as page 0, so no read leaves the page pool.  Table
+ * entries past a sequence's last used block are never read.  A length of 0
+ * gives o = 0 and lse = -inf.  No host synchronisation; asynchronous on `stream`.
+ * (Not on the pages: the page layout, the table format and the head grouping
+ * follow the common serving convention.)
+ */
+int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const int* block_table,
+                    const int* kv_lens, void* o, float* lse, int B, int H, int Hkv, int num_pages, int page_size,
+                    int max_blocks, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
+                    void* stream);
 
 /*
  * Synchronises `stream`, returns the current device's status word (FA_OK if no

@@ -33,7 +33,7 @@ def lib():
 def test_header_declares_the_entry_points():
     names = header_functions()
     for n in ("fa_forward", "fa_backward", "fa_backward_workspace_size", "fa_decode", "fa_decode_workspace_size",
-              "fa_check_status", "fa_status_string"):
+              "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_check_status", "fa_status_string"):
         assert n in names
 
 
@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 8):
+    for code in range(0, 10):
         assert fa.fa_status_string(code)
     assert "unknown" in fa.fa_status_string(99)
 
@@ -88,6 +88,37 @@ def test_decode_argument_checks(lib, args, code):
     rc = fa.fa_decode(a["q"], a["k"], a["v"], a["kv"], a["o"], a["lse"], a["B"], a["H"], a["cap"], a["d"], 0.1, 0,
                       a["ws"], a["ws_bytes"], 0)
     assert rc == code
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(bt=0), fa.FA_ERR_INVALID_ARG),
+    (dict(kv=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hkv=3), fa.FA_ERR_INVALID_ARG),       # H = 8 is not a multiple of 3
+    (dict(Hkv=0), fa.FA_ERR_INVALID_ARG),
+    (dict(ps=48), fa.FA_ERR_INVALID_ARG),       # not a power of two
+    (dict(ps=1 << 17), fa.FA_ERR_INVALID_ARG),
+    (dict(pages=0), fa.FA_ERR_INVALID_ARG),
+    (dict(blocks=0), fa.FA_ERR_INVALID_ARG),
+    (dict(kp=P + 8), fa.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=5), fa.FA_ERR_UNSUPPORTED),
+    (dict(ws=0), fa.FA_ERR_WORKSPACE),
+    (dict(ws_bytes=16), fa.FA_ERR_WORKSPACE),
+    (dict(ws=P + 16), fa.FA_ERR_WORKSPACE),
+])
+def test_decode_paged_argument_checks(lib, args, code):
+    a = dict(q=P, kp=P, vp=P, bt=P, kv=P, o=P, lse=P, B=2, H=8, Hkv=2, pages=64, ps=16, blocks=32, d=128,
+             o_dtype=0, ws=P, ws_bytes=1 << 30)
+    a.update(args)
+    rc = fa.fa_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["kv"], a["o"], a["lse"], a["B"], a["H"], a["Hkv"],
+                            a["pages"], a["ps"], a["blocks"], a["d"], 0.1, a["o_dtype"], a["ws"], a["ws_bytes"], 0)
+    assert rc == code
+
+
+def test_decode_paged_workspace_size(lib):
+    # the same partials as a contiguous decode over max_blocks * page_size keys
+    assert fa.fa_decode_paged_workspace_size(3, 8, 32, 64, 128) == fa.fa_decode_workspace_size(3, 8, 2048, 128)
+    assert fa.fa_decode_paged_workspace_size(3, 8, 0, 64, 128) == 0
 
 
 def test_decode_workspace_size(lib):
