@@ -69,6 +69,30 @@ def decode_inputs(B: int, H: int, cap: int, d: int, seed: int, len_lo: int, len_
 
 
 @dataclass
+class VarlenInputs:
+    q: torch.Tensor       # [total_q, H, d] bf16
+    k: torch.Tensor       # [total_k, H, d] bf16
+    v: torch.Tensor       # [total_k, H, d] bf16
+    cu_q: torch.Tensor    # int32 [B+1]
+    cu_k: torch.Tensor    # int32 [B+1]
+
+
+def varlen_inputs(lens_q, lens_k, H: int, d: int, seed: int) -> VarlenInputs:
+    """Packed batch: sequence b has lens_q[b] queries and lens_k[b] keys.  Draw order:
+    Q, K, V of the packed tensors, N(0,1), bf16."""
+    gen = torch.Generator("cpu").manual_seed(seed)
+    cu_q = torch.zeros(len(lens_q) + 1, dtype=torch.int32)
+    cu_k = torch.zeros(len(lens_k) + 1, dtype=torch.int32)
+    cu_q[1:] = torch.cumsum(torch.tensor(lens_q, dtype=torch.int64), 0).to(torch.int32)
+    cu_k[1:] = torch.cumsum(torch.tensor(lens_k, dtype=torch.int64), 0).to(torch.int32)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    q = _normal(gen, (tq, H, d)).to(torch.bfloat16)
+    k = _normal(gen, (tk, H, d)).to(torch.bfloat16)
+    v = _normal(gen, (tk, H, d)).to(torch.bfloat16)
+    return VarlenInputs(q, k, v, cu_q, cu_k)
+
+
+@dataclass
 class PagedDecodeInputs:
     q: torch.Tensor            # [B, H, d] bf16
     kpages: torch.Tensor       # [num_pages, Hkv, page_size, d] bf16
@@ -118,6 +142,8 @@ WORKLOADS = {
     "decode_cap32768": dict(kind="decode", B=64, H=32, cap=32768, d=128, len_lo=1024, len_hi=32768, seed=5),
     # Paged cache with grouped heads: the same batch and lengths as the decode workload,
     # 8 KV heads shared by groups of 4 query heads, 64-token pages in shuffled order.
+    # Packed prefill batch of 16 causal sequences of 512 to 8,192 tokens.
+    "prefill_varlen": dict(kind="varlen", B=16, H=16, d=128, len_lo=512, len_hi=8192, causal=True, seed=7),
     "decode_paged_gqa": dict(kind="decode_paged", B=64, H=32, Hkv=8, page_size=64, max_blocks=512, d=128,
                              len_lo=1024, len_hi=32768, seed=6),
 }

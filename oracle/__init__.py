@@ -60,6 +60,9 @@ def _load():
                                         ctypes.c_double, c_int]
         lib.oracle_decode.restype = None
         lib.oracle_decode.argtypes = [vp, vp, vp, c_int, vp, dp, dp, i64, i64, i64, i64, ctypes.c_double]
+        lib.oracle_forward_varlen.restype = None
+        lib.oracle_forward_varlen.argtypes = [vp, vp, vp, c_int, dp, dp, vp, vp, i64, i64, i64, i64, ctypes.c_double,
+                                              c_int]
         lib.oracle_decode_paged.restype = c_int
         lib.oracle_decode_paged.argtypes = [vp, vp, vp, c_int, vp, vp, dp, dp, i64, i64, i64, i64, i64, i64, i64,
                                             ctypes.c_double]
@@ -189,6 +192,27 @@ def decode(q, kcache, vcache, kv_lens, scale: float):
     lse = np.empty((B, H), np.float64)
     _load().oracle_decode(pq, pk, pv, dt, lens.ctypes.data, o.ctypes.data, lse.ctypes.data, B, H, cap, d,
                           float(scale))
+    return o, lse
+
+
+def forward_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
+    """Packed variable-length forward: q [total_q,H,d], k/v [total_k,H,d], cu_q/cu_k int32 [B+1].
+    Returns O [total_q,H,d] and LSE [H,total_q] in float64."""
+    total_q, H, d = q.shape
+    kq, pq, cq = _as_input(q)
+    kk, pk, ck = _as_input(k)
+    kv, pv, cv = _as_input(v)
+    dt = _same_kind(cq, ck, cv)
+    cq_ = np.ascontiguousarray(np.asarray(cu_q, dtype=np.int32))
+    ck_ = np.ascontiguousarray(np.asarray(cu_k, dtype=np.int32))
+    B = cq_.shape[0] - 1
+    if ck_.shape != cq_.shape or cq_[0] != 0 or ck_[0] != 0 or cq_[-1] != total_q or ck_[-1] != k.shape[0] \
+            or np.any(np.diff(cq_) < 0) or np.any(np.diff(ck_) < 0):
+        raise ValueError("cu_seqlens must start at 0, be non-decreasing and end at the packed lengths")
+    o = np.empty((total_q, H, d), np.float64)
+    lse = np.empty((H, total_q), np.float64)
+    _load().oracle_forward_varlen(pq, pk, pv, dt, o.ctypes.data, lse.ctypes.data, cq_.ctypes.data, ck_.ctypes.data,
+                                  B, H, total_q, d, float(scale), int(bool(causal)))
     return o, lse
 
 

@@ -137,6 +137,62 @@ void oracle_forward(const void* q, const void* k, const void* v, int dtype,
 }
 
 /*
+ * Forward pass over a packed batch of sequences of different lengths.  The
+ * pages' problem statement is per sequence ([W] "The problem it solves"; [L]
+ * "Basic Flash Attention Forward Pass" gives one (B, H, L, D) batch); packing
+ * sequences of different lengths end to end is not on the pages.  Sequence b
+ * owns query rows [cu_q[b], cu_q[b+1]) and key rows [cu_k[b], cu_k[b+1]) of the
+ * packed tensors q [total_q, H, d] and k, v [total_k, H, d]; each sequence is
+ * attended to on its own, exactly as oracle_forward with Lq = cu_q[b+1] - cu_q[b]
+ * and Lk = cu_k[b+1] - cu_k[b] (bottom-right causal alignment).
+ * Outputs o [total_q, H, d] and lse [H, total_q].
+ */
+void oracle_forward_varlen(const void* q, const void* k, const void* v, int dtype, double* o, double* lse,
+                           const int32_t* cu_q, const int32_t* cu_k, int64_t B, int64_t H, int64_t total_q,
+                           int64_t d, double scale, int causal) {
+    int64_t max_k = 1;
+    for (int64_t b = 0; b < B; ++b)
+        if (cu_k[b + 1] - cu_k[b] > max_k) max_k = cu_k[b + 1] - cu_k[b];
+    const int64_t rows = total_q * H;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)max_k);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            const int64_t h = r % H, row = r / H;  // packed row, head
+            int64_t b = 0;
+            while (b + 1 < B && cu_q[b + 1] <= row) ++b;
+            const int64_t Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+            const int64_t i = row - cu_q[b];
+            const int64_t n = oracle_permitted_keys(i, Lq, Lk, causal);
+            double* orow = o + (row * H + h) * d;
+            for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+            if (n <= 0) {
+                lse[h * total_q + row] = -INFINITY;
+                continue;
+            }
+            double M = -INFINITY;
+            for (int64_t j = 0; j < n; ++j) {
+                const int64_t krow = ((cu_k[b] + j) * H + h) * d;
+                double sdot = 0.0;
+                for (int64_t c = 0; c < d; ++c) sdot += elem(q, (row * H + h) * d + c, dtype) * elem(k, krow + c, dtype);
+                t[j] = scale * sdot;
+                if (t[j] > M) M = t[j];
+            }
+            double Z = 0.0;
+            for (int64_t j = 0; j < n; ++j) Z += exp(t[j] - M);
+            for (int64_t j = 0; j < n; ++j) {
+                const double pj = exp(t[j] - M) / Z;
+                const int64_t vrow = ((cu_k[b] + j) * H + h) * d;
+                for (int64_t c = 0; c < d; ++c) orow[c] += pj * elem(v, vrow + c, dtype);
+            }
+            lse[h * total_q + row] = M + log(Z);
+        }
+        free(t);
+    }
+}
+
+/*
  * Forward pass on a chosen set of rows.  rows[s] is a flat row index
  * (b*H + h)*Lq + i; the result for it goes to o_out[s*d ...] and lse_out[s].
  * Row sampling is exact: each row of the output depends on that query row

@@ -351,3 +351,55 @@ def test_paged_decode_unused_slots_and_errors():
         oracle.decode_paged(q, kp, vp, t3, lens, 0.5)
     with pytest.raises(ValueError):
         oracle.decode_paged(torch.randn(B, 3, d).to(torch.bfloat16), kp, vp, table, lens, 0.5)
+
+
+# ----------------------------------------------------------------------------- packed variable-length forward
+def _pack(seqs):
+    """[L_b, H, d] tensors -> packed [sum L_b, H, d] and cu_seqlens [B+1]."""
+    cu = np.zeros(len(seqs) + 1, np.int32)
+    cu[1:] = np.cumsum([s.shape[0] for s in seqs])
+    return torch.cat(seqs, 0), cu
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_forward_equals_per_sequence_forward(causal):
+    """Each packed sequence is attended to on its own: equal to the batched oracle
+    run on that sequence alone (chunked prefill: Lq < Lk, bottom-right causal)."""
+    g = torch.Generator("cpu").manual_seed(21)
+    H, d = 3, 8
+    lq = [5, 1, 0, 17, 9]
+    lk = [5, 4, 3, 25, 9] if causal else [7, 1, 2, 11, 9]
+    qs = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lq]
+    ks = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lk]
+    vs = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lk]
+    q, cq = _pack(qs)
+    k, ck = _pack(ks)
+    v, _ = _pack(vs)
+    o, lse = oracle.forward_varlen(q, k, v, cq, ck, 0.35, causal)
+    for b in range(len(lq)):
+        if lq[b] == 0:
+            continue
+        ob, lb = oracle.forward(qs[b].permute(1, 0, 2)[None].contiguous(), ks[b].permute(1, 0, 2)[None].contiguous(),
+                                vs[b].permute(1, 0, 2)[None].contiguous(), 0.35, causal)
+        assert np.max(np.abs(o[cq[b]:cq[b + 1]] - ob[0].transpose(1, 0, 2))) <= 1e-12
+        assert np.max(np.abs(lse[:, cq[b]:cq[b + 1]] - lb[0])) <= 1e-12
+
+
+def test_varlen_forward_repacking_permutes_outputs():
+    g = torch.Generator("cpu").manual_seed(22)
+    H, d = 2, 4
+    lens = [3, 6, 2]
+    qs = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lens]
+    ks = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lens]
+    vs = [torch.randn(n, H, d, generator=g).to(torch.bfloat16) for n in lens]
+    q, cu = _pack(qs)
+    o, lse = oracle.forward_varlen(q, _pack(ks)[0], _pack(vs)[0], cu, cu, 0.5, True)
+    order = [2, 0, 1]
+    q2, cu2 = _pack([qs[i] for i in order])
+    o2, lse2 = oracle.forward_varlen(q2, _pack([ks[i] for i in order])[0], _pack([vs[i] for i in order])[0],
+                                     cu2, cu2, 0.5, True)
+    for new_b, b in enumerate(order):
+        assert np.array_equal(o2[cu2[new_b]:cu2[new_b + 1]], o[cu[b]:cu[b + 1]])
+        assert np.array_equal(lse2[:, cu2[new_b]:cu2[new_b + 1]], lse[:, cu[b]:cu[b + 1]])
+    with pytest.raises(ValueError):
+        oracle.forward_varlen(q, _pack(ks)[0], _pack(vs)[0], np.array([0, 5, 4, 11], np.int32), cu, 0.5, True)
