@@ -435,6 +435,34 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "traffic": recorded_traffic("fa_decode", "decode_cap32768", ["decode_sm100.cu"])}
     del kc, vc
 
+    # packed prefill batch of sequences of different lengths (causal)
+    w = WORKLOADS["prefill_varlen"]
+    Bv, Hv, dv_ = w["B"], w["H"], w["d"]
+    cg = torch.Generator("cpu").manual_seed(w["seed"])
+    lens_v = torch.randint(w["len_lo"], w["len_hi"] + 1, (Bv,), generator=cg).to(torch.int32)
+    cu = torch.zeros(Bv + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens_v, 0)
+    tot = int(cu[-1])
+    qv, kv_, vv = (torch.randn(tot, Hv, dv_, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+    ov = torch.empty(tot, Hv, dv_, dtype=torch.float32, device=device)
+    lv = torch.empty(Hv, tot, dtype=torch.float32, device=device)
+    cu_d = cu.to(device)
+    mx = int(lens_v.max())
+    sc_v = 1.0 / math.sqrt(dv_)
+
+    def fwd_varlen():
+        rc = fa.fa_forward_varlen(qv, kv_, vv, ov, lv, cu_d, cu_d, Bv, Hv, tot, tot, mx, dv_, sc_v, 1, fa.FA_DT_F32,
+                                  stream)
+        assert rc == fa.FA_OK
+
+    fv = sum(attn_flops(1, Hv, int(n), int(n), dv_, True) for n in lens_v)
+    t_v = time_steps(fwd_varlen, steps, warm, stream, dist, device) / steps
+    legs["prefill_varlen"] = {"ms": round(t_v * 1e3, 4), "TFLOP/s": round(fv / t_v / 1e12, 1),
+                              "frac_of_peak": round(fv / t_v / 1e12 / peaks["bf16_tflops"], 4), "launches": 1,
+                              "config": "16 causal sequences, lengths U[512, 8192] (%d tokens), H16 d128, packed"
+                                        % tot}
+    del qv, kv_, vv, ov, lv
+
     # paged cache with grouped heads: same batch and lengths, 8 KV heads for 32 query heads
     w = WORKLOADS["decode_paged_gqa"]
     B, H, Hkv, ps, nblk, d = w["B"], w["H"], w["Hkv"], w["page_size"], w["max_blocks"], w["d"]

@@ -37,6 +37,7 @@ FA_ERR_DEVICE = 6
 FA_ERR_KV_LEN = 7
 FA_ERR_TOO_LARGE = 8
 FA_ERR_PAGE = 9
+FA_ERR_SEQLEN = 10
 FA_NOALLOC_MAX_ROWS = 1 << 20
 FA_DT_BF16 = 0
 FA_DT_F32 = 1
@@ -74,6 +75,8 @@ def load_library():
     lib.fa_decode_workspace_size.argtypes = [i, i, i, i]
     lib.fa_decode.restype = i
     lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
+    lib.fa_forward_varlen.restype = i
+    lib.fa_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
     lib.fa_decode_paged_workspace_size.restype = sz
     lib.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_decode_paged.restype = i
@@ -140,6 +143,13 @@ def fa_decode(q, kcache, vcache, kv_lens, o, lse, B, H, cap, d, scale, o_dtype, 
     return load_library().fa_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(kv_lens), _ptr(o), _ptr(lse), B,
                                     H, cap, d, float(scale), int(o_dtype), _ptr(workspace), int(workspace_bytes),
                                     _stream(stream))
+
+
+def fa_forward_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, max_seqlen_q, d, scale,
+                      causal, o_dtype, stream=None) -> int:
+    return load_library().fa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                                            _ptr(cu_seqlens_k), B, H, total_q, total_k, max_seqlen_q, d, float(scale),
+                                            int(causal), int(o_dtype), _stream(stream))
 
 
 def fa_decode_paged_workspace_size(B, H, max_blocks, page_size, d) -> int:
@@ -255,4 +265,25 @@ def decode_paged(q, kpages, vpages, block_table, kv_lens, scale=None, out_dtype=
     rc = fa_decode_paged(q, kpages, vpages, block_table, kv_lens, o, lse, B, H, Hkv, num_pages, page_size, max_blocks,
                          d, scale, _DT[out_dtype], ws, ws.numel() * ws.element_size(), stream)
     _check(rc, "fa_decode_paged")
+    return o, lse
+
+
+def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, scale=None, causal=False,
+                   out_dtype=torch.float32, stream=None):
+    """Packed batch: q [total_q,H,d], k/v [total_k,H,d] (bf16), cu_seqlens int32 [B+1] (device).
+    Returns o [total_q,H,d] (out_dtype) and lse [H,total_q] (fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    _need(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _need(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.shape[0] - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty((total_q, H, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device)
+    rc = fa_forward_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, int(max_seqlen_q), d,
+                           scale, causal, _DT[out_dtype], stream)
+    _check(rc, "fa_forward_varlen")
     return o, lse

@@ -103,6 +103,23 @@ int encode_out_map_impl(CUtensorMap* map, void* base, int BH, int L, int d, int 
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// A packed token-major tensor [total, H, d] (bf16 or fp32) as a 3-D TMA map
+// {d, H, total} with boxes of 128 bytes x 1 head x box_rows tokens, so a box
+// lands in shared memory exactly like a batched [rows][128 bytes] box.
+// 128-byte swizzle.  Rows past total read as zero / are clipped on stores.
+int encode_packed_map_impl(CUtensorMap* map, const void* base, int total, int H, int d, int box_rows,
+                           int elem_bytes) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(total)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem_bytes, static_cast<cuuint64_t>(H) * d * elem_bytes};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), 1, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(map, elem_bytes == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 bool dims_ok(int B, int H, int L, int d) {
     if (B <= 0 || H <= 0 || L <= 0) return false;
     const long long bh = static_cast<long long>(B) * H;
@@ -127,6 +144,10 @@ bool shape_ok(int B, int H, int L, int d) { return dims_ok(B, H, L, d); }
 int encode_out_map(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype) {
     return encode_out_map_impl(map, base, BH, L, d, o_dtype);
 }
+int encode_packed_map(CUtensorMap* map, const void* base, int total, int H, int d, int box_rows, int elem_bytes,
+                      bool) {
+    return encode_packed_map_impl(map, base, total, H, d, box_rows, elem_bytes);
+}
 
 }  // namespace fa
 
@@ -148,6 +169,8 @@ const char* fa_status_string(int status) {
             return "FA_ERR_TOO_LARGE: B*H*Lq exceeds FA_NOALLOC_MAX_ROWS, the fixed scratch of fa_backward_noalloc";
         case FA_ERR_PAGE:
             return "FA_ERR_PAGE: a block-table entry used by a valid key was outside [0, num_pages) (read as page 0)";
+        case FA_ERR_SEQLEN:
+            return "FA_ERR_SEQLEN: a packed sequence's offsets or lengths were invalid; its rows were skipped";
         default: return "unknown fa_status";
     }
 }
@@ -286,6 +309,53 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o, cons
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
     cudaError_t e = launch_bwd(p, d, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                      const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q, int d,
+                      float scale, int causal, int o_dtype, void* stream) {
+    if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (B <= 0 || H <= 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+        !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+        return FA_ERR_INVALID_ARG;
+    if (static_cast<long long>(total_q) * H > 0x7FFFFFFFLL || static_cast<long long>(total_k) * H > 0x7FFFFFFFLL)
+        return FA_ERR_INVALID_ARG;
+    const long long max_pairs = (static_cast<long long>(max_seqlen_q) + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    if (static_cast<long long>(B) * H * max_pairs > 0x7FFFFFFFLL || max_pairs * kFwdRowsPerCta > 0x7FFFFFFFLL)
+        return FA_ERR_INVALID_ARG;
+    if (total_q == 0 || max_pairs == 0) return FA_OK;
+    if (total_k == 0) return FA_ERR_INVALID_ARG;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    FwdParams p{};
+    if ((rc = encode_packed_map_impl(&p.tm_q, q, total_q, H, d, kFwdBM, 2)) != FA_OK) return rc;
+    if ((rc = encode_packed_map_impl(&p.tm_k, k, total_k, H, d, kFwdBN, 2)) != FA_OK) return rc;
+    if ((rc = encode_packed_map_impl(&p.tm_v, v, total_k, H, d, kFwdBN, 2)) != FA_OK) return rc;
+    if ((rc = encode_packed_map_impl(&p.tm_o, o, total_q, H, d, 32, o_dtype == FA_DT_F32 ? 4 : 2)) != FA_OK)
+        return rc;
+    p.o = o;
+    p.lse = lse;
+    p.status = st->status_ptr;
+    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    p.cu_q = cu_seqlens_q;
+    p.cu_k = cu_seqlens_k;
+    p.max_pairs = static_cast<int>(max_pairs);
+    p.B = B;
+    p.H = H;
+    p.Lq = total_q;
+    p.Lk = total_k;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.o_dtype = o_dtype;
+    cudaError_t e = launch_fwd_varlen(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

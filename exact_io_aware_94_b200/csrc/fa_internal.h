@@ -37,6 +37,12 @@ struct __align__(64) FwdParams {
     float* lse;
     int* status;
     unsigned int* sched;  // [0]: next unit ticket, [1]: CTAs finished; both zero between launches
+    // packed variable-length batch (fa_forward_varlen): sequence b owns rows [cu_q[b], cu_q[b+1])
+    // of q, o [total_q, H, d] and [cu_k[b], cu_k[b+1]) of k, v [total_k, H, d]; Lq = total_q,
+    // Lk = total_k, and max_pairs = ceil(max_seqlen_q / 256).  Null for a batched call.
+    const int* cu_q;
+    const int* cu_k;
+    int max_pairs;
     int B, H, Lq, Lk;
     float scale;       // multiplies q.k
     float scale_log2;  // scale * log2(e)
@@ -103,6 +109,9 @@ cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaS
 
 int fwd_smem_bytes(int d);
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
+cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
+int encode_packed_map(CUtensorMap* map, const void* base, int total, int H, int d, int box_rows, int elem_bytes,
+                      bool swizzle_box64);
 int encode_out_map(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype);
 
 }  // namespace fa

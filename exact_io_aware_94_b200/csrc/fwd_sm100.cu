@@ -74,9 +74,11 @@ struct FwdLayout {
     static constexpr int kBytes = kStageOff + 8 * 4096 + 1024;  // + alignment slack
 };
 
-// One work unit: which (b*H + h), which pair of 128-row tiles, how many KV tiles each needs.
+// One work unit: which (b*H + h), which pair of 128-row tiles, how many KV tiles each needs,
+// and where its sequence lives (packed first rows and lengths; 0, 0, Lq, Lk for a batched call).
 struct Unit {
     int bh, i0, n_kv0, n_kv1;
+    int q0, k0, lq, lk;
 };
 
 // Units in a fixed global order: longest causal rows first (pair index
@@ -105,10 +107,60 @@ __device__ __forceinline__ Unit unit_of(const FwdParams& p, int u) {
     }
     r.n_kv0 = n[0];
     r.n_kv1 = n[1];
+    r.q0 = 0;
+    r.k0 = 0;
+    r.lq = p.Lq;
+    r.lk = p.Lk;
     return r;
 }
 
-template <int D>
+// Packed variable-length batch: unit u is (pair, b*H + h) in a virtual space of
+// max_pairs pairs per (b, h), longest causal rows first.  Units past a
+// sequence's end are empty (no KV tiles).  A sequence whose offsets are out of
+// range or decreasing, that is longer than max_pairs * 256 rows, that has
+// queries but no keys, or (causal) more queries than keys is skipped and
+// flagged FA_ERR_SEQLEN (once, by the producer, from its pair-0 unit).
+__device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u, bool flag) {
+    const int BH = p.B * p.H;
+    Unit r;
+    const int pair = p.max_pairs - 1 - u / BH;
+    r.bh = u % BH;
+    r.i0 = pair * kFwdRowsPerCta;
+    r.n_kv0 = 0;
+    r.n_kv1 = 0;
+    const int b = r.bh / p.H;
+    const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+    r.q0 = q0;
+    r.k0 = k0;
+    r.lq = q1 - q0;
+    r.lk = k1 - k0;
+    const bool bad = q0 < 0 || q1 < q0 || q1 > p.Lq || k0 < 0 || k1 < k0 || k1 > p.Lk ||
+                     r.lq > p.max_pairs * kFwdRowsPerCta || (r.lq > 0 && r.lk == 0) || (p.causal && r.lq > r.lk);
+    if (bad) {
+        if (flag && pair == 0) atomicCAS(p.status, 0, FA_ERR_SEQLEN);
+        r.lq = 0;
+        return r;
+    }
+    const int n_kv_all = (r.lk + kFwdBN - 1) / kFwdBN;
+    const int off = r.lk - r.lq;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const int first = r.i0 + w * kFwdBM;
+        int n = 0;
+        if (first < r.lq)
+            n = p.causal ? min(n_kv_all, (min(first + kFwdBM - 1, r.lq - 1) + off) / kFwdBN + 1) : n_kv_all;
+        if (w == 0) r.n_kv0 = n; else r.n_kv1 = n;
+    }
+    return r;
+}
+
+template <bool VARLEN>
+__device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag) {
+    if constexpr (VARLEN) return unit_of_varlen(p, u, flag);
+    else return unit_of(p, u);
+}
+
+template <int D, bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using Lay = FwdLayout<D>;
     constexpr int S = Lay::kStages;
@@ -141,8 +193,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = p.B * p.H * ((p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
-    const int off = p.Lk - p.Lq;
+    const int n_units = p.B * p.H * (VARLEN ? p.max_pairs : (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
 
     // ---- setup
     if (threadIdx.x == 0) {
@@ -205,16 +256,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 // claim the next unit (heavy-first order) and publish it
                 const int rs = it % kUnitRing;
                 if (it >= kUnitRing && !(ok = wait(&bar_ufree[rs], ((it / kUnitRing) - 1) & 1))) break;
-                unsigned int ticket = 0;
-                if (lane == 0) ticket = atomicAdd(p.sched, 1u);
-                const int u = static_cast<int>(min(__shfl_sync(0xffffffffu, ticket, 0), static_cast<unsigned>(n_units)));
+                int u;
+                Unit un;
+                for (;;) {  // a packed batch's virtual units past a sequence's end are skipped here
+                    unsigned int ticket = 0;
+                    if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+                    u = static_cast<int>(min(__shfl_sync(0xffffffffu, ticket, 0), static_cast<unsigned>(n_units)));
+                    if (u >= n_units) break;
+                    un = get_unit<VARLEN>(p, u, true);
+                    if (!VARLEN || un.n_kv0 > 0 || un.n_kv1 > 0) break;
+                }
                 if (lane == 0) {
                     s_unit[rs] = u;
                     mbar_arrive(&bar_ufull[rs]);
                 }
                 __syncwarp();
                 if (u >= n_units) break;
-                const Unit un = unit_of(p, u);
                 const int n_max = max(un.n_kv0, un.n_kv1);
                 // Q_w as soon as warpgroup w's S MMAs of its previous unit are done with the
                 // buffer (under a causal mask warpgroup 0 lets go of it a tile earlier).
@@ -222,9 +279,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 auto load_q = [&](int w) -> bool {
                     if (q_iter[w] > 0 && !wait(&bar_q_free[w], (q_iter[w] - 1) & 1)) return false;
                     mbar_arrive_expect_tx_w(&bar_q[w], Lay::kTileBytes);
+                    // batched maps are [B*H][L][d]; packed maps are [total][H][d]
+                    const int cy = VARLEN ? un.bh % p.H : un.i0 + w * kFwdBM;
+                    const int cz = VARLEN ? un.q0 + un.i0 + w * kFwdBM : un.bh;
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d_w(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, &bar_q[w], b * 64,
-                                      un.i0 + w * kFwdBM, un.bh);
+                        tma_load_3d_w(sQ + w * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_q, &bar_q[w], b * 64, cy,
+                                      cz);
                     ++q_iter[w];
                     return true;
                 };
@@ -232,17 +292,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 for (int j = 0; j < n_max; ++j, ++kc) {
                     const int s = kc % S;
                     if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
+                    const int ky = VARLEN ? un.bh % p.H : j * kFwdBN;
+                    const int kz = VARLEN ? un.k0 + j * kFwdBN : un.bh;
                     mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
-                                    j * kFwdBN, un.bh);
+                        tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64, ky,
+                                      kz);
                     ++nk;
                     if (j == 0 && un.n_kv1 > 0 && !(ok = load_q(1))) break;
                     if (kc >= S && !(ok = wait(&bar_vfree[s], ((kc / S) - 1) & 1))) break;
                     mbar_arrive_expect_tx_w(&bar_v[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d_w(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64,
-                                    j * kFwdBN, un.bh);
+                        tma_load_3d_w(sV + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_v, &bar_v[s], b * 64, ky,
+                                      kz);
                     ++nv;
                 }
             }
@@ -300,7 +362,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
-                const Unit un = unit_of(p, u);
+                const Unit un = get_unit<VARLEN>(p, u, false);
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
@@ -386,12 +448,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit un = unit_of(p, u);
+            const Unit un = get_unit<VARLEN>(p, u, false);
             const int n = (w == 0) ? un.n_kv0 : un.n_kv1;
             if (n == 0) continue;
             const int tile_first_row = un.i0 + w * kFwdBM;
             const int row = tile_first_row + row_in_tile;
-            const int limit = p.causal ? min(row + off, p.Lk - 1) : p.Lk - 1;  // highest permitted key
+            const int off = un.lk - un.lq;  // causal: query i sits at key position i + off
+            const int limit = p.causal ? min(row + off, un.lk - 1) : un.lk - 1;  // highest permitted key
 
             float m_ref = -INFINITY;  // running max of raw scores q.k (reference for P~)
             float l = 0.0f;           // running sum of the unrounded P~: gives the LSE
@@ -414,7 +477,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 }
                 const int kv0 = j * kFwdBN;
                 const bool need_mask =
-                    (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) || (kv0 + kFwdBN > p.Lk);
+                    (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) || (kv0 + kFwdBN > un.lk);
                 if (need_mask) {
 #pragma unroll
                     for (int c = 0; c < kFwdBN; ++c)
@@ -517,12 +580,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
                 const bool f32 = p.o_dtype == FA_DT_F32;
                 const int n_chunks = f32 ? D / 32 : D / 64;
+                // A packed sequence's last partial 32-row box would spill into the next
+                // sequence's rows: its rows are written one by one instead.
+                const bool by_rows = VARLEN && tile_first_row + wq * 32 + 32 > un.lq;
+                const size_t tok_bytes = static_cast<size_t>(p.H) * D * (f32 ? 4 : 2);
+                uint8_t* orow = static_cast<uint8_t*>(p.o) + static_cast<size_t>(un.q0 + row) * tok_bytes +
+                                static_cast<size_t>(un.bh % p.H) * D * (f32 ? 4 : 2);
 #pragma unroll
                 for (int k = 0; k < D / 32; ++k) {
                     if (k >= n_chunks) break;
                     // the stage's previous tile store has finished reading it
-                    if (lane == 0) bulk_wait_group_read0();
-                    __syncwarp();
+                    if (!by_rows) {
+                        if (lane == 0) bulk_wait_group_read0();
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         uint4 v;
@@ -539,17 +610,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                             v.z = pack_bf16x2(__uint_as_float(ov[c0 + 4]) * inv_l, __uint_as_float(ov[c0 + 5]) * inv_l);
                             v.w = pack_bf16x2(__uint_as_float(ov[c0 + 6]) * inv_l, __uint_as_float(ov[c0 + 7]) * inv_l);
                         }
-                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
+                        if (by_rows) {
+                            if (row < un.lq) *reinterpret_cast<uint4*>(orow + k * 128 + q * 16) = v;
+                        } else {
+                            *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
+                        }
                     }
+                    if (by_rows) continue;
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (tile_first_row + wq * 32 < p.Lq)
-                            tma_store_3d(&p.tm_o, stg, k * (f32 ? 32 : 64), tile_first_row + wq * 32, un.bh);
+                        if constexpr (VARLEN) {
+                            tma_store_3d(&p.tm_o, stg, k * (f32 ? 32 : 64), un.bh % p.H, un.q0 + tile_first_row + wq * 32);
+                        } else {
+                            if (tile_first_row + wq * 32 < p.Lq)
+                                tma_store_3d(&p.tm_o, stg, k * (f32 ? 32 : 64), tile_first_row + wq * 32, un.bh);
+                        }
                         bulk_commit_group();
                     }
                 }
-                if (row < p.Lq) p.lse[static_cast<size_t>(un.bh) * p.Lq + row] = m_ref * p.scale + logf(l);
+                if (row < un.lq) {
+                    const size_t li = VARLEN ? static_cast<size_t>(un.bh % p.H) * p.Lq + un.q0 + row
+                                             : static_cast<size_t>(un.bh) * p.Lq + row;
+                    p.lse[li] = m_ref * p.scale + logf(l);
+                }
             }
         }
     }
@@ -590,25 +674,28 @@ cudaError_t check_register_split(K kernel) {
 
 int fwd_smem_bytes(int d) { return d == 128 ? FwdLayout<128>::kBytes : FwdLayout<64>::kBytes; }
 
-cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
-    const long long units = static_cast<long long>(p.B) * p.H * ((p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+template <int D, bool VARLEN>
+cudaError_t launch_fwd_kernel(const FwdParams& p, int num_sms, cudaStream_t stream) {
+    const long long pairs = VARLEN ? p.max_pairs : (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    const long long units = static_cast<long long>(p.B) * p.H * pairs;
+    if (units == 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
-    const int smem = fwd_smem_bytes(d);
+    const int smem = fwd_smem_bytes(D);
     cudaError_t e;
-    if (d == 128) {
-        if ((e = check_register_split(fa_fwd_kernel<128>)) != cudaSuccess) return e;
-        if ((e = cudaFuncSetAttribute(fa_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-            cudaSuccess)
-            return e;
-        fa_fwd_kernel<128><<<grid, kFwdThreads, smem, stream>>>(p);
-    } else {
-        if ((e = check_register_split(fa_fwd_kernel<64>)) != cudaSuccess) return e;
-        if ((e = cudaFuncSetAttribute(fa_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-            cudaSuccess)
-            return e;
-        fa_fwd_kernel<64><<<grid, kFwdThreads, smem, stream>>>(p);
-    }
+    if ((e = check_register_split(fa_fwd_kernel<D, VARLEN>)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(fa_fwd_kernel<D, VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    fa_fwd_kernel<D, VARLEN><<<grid, kFwdThreads, smem, stream>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
+    return d == 128 ? launch_fwd_kernel<128, false>(p, num_sms, stream) : launch_fwd_kernel<64, false>(p, num_sms, stream);
+}
+
+cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
+    return d == 128 ? launch_fwd_kernel<128, true>(p, num_sms, stream) : launch_fwd_kernel<64, true>(p, num_sms, stream);
 }
 
 }  // namespace fa

@@ -59,7 +59,8 @@ typedef enum {
     FA_ERR_DEVICE = 6,      /* current device is not compute capability 10.0 */
     FA_ERR_KV_LEN = 7,      /* device: a decode cache length was outside [0, cap] (clamped) */
     FA_ERR_TOO_LARGE = 8,   /* problem larger than the fixed scratch of fa_backward_noalloc */
-    FA_ERR_PAGE = 9         /* device: a block-table entry used by a valid key was outside [0, num_pages) */
+    FA_ERR_PAGE = 9,        /* device: a block-table entry used by a valid key was outside [0, num_pages) */
+    FA_ERR_SEQLEN = 10      /* device: a packed sequence's offsets or lengths were invalid (sequence skipped) */
 } fa_status;
 
 enum { FA_DT_BF16 = 0, FA_DT_F32 = 1 };
@@ -142,6 +143,31 @@ size_t fa_decode_workspace_size(int B, int H, int cap, int d);
 int fa_decode(const void* q, const void* kcache, const void* vcache, const int* kv_lens, void* o, float* lse,
               int B, int H, int cap, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
               void* stream);
+
+/*
+ * Forward pass over a packed batch of sequences of different lengths (the
+ * prefill of a batch of prompts; chunked prefill when a sequence's queries are
+ * the last Lq of its Lk keys).  Each sequence is attended to on its own with
+ * the same computation as fa_forward ("What FlashAttention does instead",
+ * "The Three Running Statistics"); packing sequences end to end is not on the
+ * pages.
+ *   q [total_q, H, d], k, v [total_k, H, d] (bf16, token-major: row t holds all
+ *   heads of token t); cu_seqlens_q, cu_seqlens_k int32 [B+1] on the device:
+ *   sequence b owns query rows [cu_q[b], cu_q[b+1]) and key rows
+ *   [cu_k[b], cu_k[b+1]), with cu[0] = 0 and cu[B] = total.
+ *   max_seqlen_q >= every cu_q[b+1] - cu_q[b] (it sizes the work).
+ *   o [total_q, H, d] (o_dtype), lse [H, total_q] fp32.
+ * Causal masking is bottom-right per sequence (query i of a sequence sits at
+ * key position i + Lk_b - Lq_b) and needs Lq_b <= Lk_b.  q, k, v, o must be
+ * 16-byte aligned.  total_q = 0 returns FA_OK without a launch.  On the
+ * device, a sequence whose offsets are out of range or decreasing, that is
+ * longer than max_seqlen_q rounded up to 256, that has queries but no keys, or
+ * (causal) more queries than keys is skipped (its rows are not written) and
+ * flagged FA_ERR_SEQLEN in the status word.  Asynchronous on `stream`.
+ */
+int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
+                      const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q, int d,
+                      float scale, int causal, int o_dtype, void* stream);
 
 /*
  * Workspace bytes fa_decode_paged needs: the same split-KV partials as

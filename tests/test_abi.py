@@ -33,7 +33,8 @@ def lib():
 def test_header_declares_the_entry_points():
     names = header_functions()
     for n in ("fa_forward", "fa_backward", "fa_backward_workspace_size", "fa_decode", "fa_decode_workspace_size",
-              "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_check_status", "fa_status_string"):
+              "fa_decode_paged", "fa_decode_paged_workspace_size", "fa_forward_varlen", "fa_check_status",
+              "fa_status_string"):
         assert n in names
 
 
@@ -44,7 +45,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 10):
+    for code in range(0, 11):
         assert fa.fa_status_string(code)
     assert "unknown" in fa.fa_status_string(99)
 
@@ -119,6 +120,26 @@ def test_decode_paged_workspace_size(lib):
     # the same partials as a contiguous decode over max_blocks * page_size keys
     assert fa.fa_decode_paged_workspace_size(3, 8, 32, 64, 128) == fa.fa_decode_workspace_size(3, 8, 2048, 128)
     assert fa.fa_decode_paged_workspace_size(3, 8, 0, 64, 128) == 0
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(cq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(q=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(B=0), fa.FA_ERR_INVALID_ARG),
+    (dict(tq=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(tk=0), fa.FA_ERR_INVALID_ARG),
+    (dict(k=P + 4), fa.FA_ERR_INVALID_ARG),
+    (dict(o_dtype=3), fa.FA_ERR_UNSUPPORTED),
+    (dict(tq=0), fa.FA_OK),            # nothing to do: no launch
+    (dict(maxq=0), fa.FA_OK),
+])
+def test_forward_varlen_argument_checks(lib, args, code):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cq=P, ck=P, B=3, H=4, tq=100, tk=120, maxq=64, d=128, o_dtype=0)
+    a.update(args)
+    rc = fa.fa_forward_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"], a["B"], a["H"], a["tq"],
+                              a["tk"], a["maxq"], a["d"], 0.1, 1, a["o_dtype"], 0)
+    assert rc == code
 
 
 def test_decode_workspace_size(lib):
