@@ -511,7 +511,9 @@ def run_profile_case(args, device):
     """One path of the library, W + K calls on seeded device inputs, for a profiler
     (ncu) to capture; prints a single status line.  fwd: the headline forward;
     bwd: forward then backward at the 8,192-token training shape; decode_small:
-    decode at B=16 H=32 cap=8192 (1 GiB of cache, small enough to capture)."""
+    decode at B=16 H=32 cap=8192 (1 GiB of cache, small enough to capture);
+    varlen_small: packed causal forward of 8 sequences of 512..4,096 tokens;
+    decode_paged_small: paged, grouped-head decode at B=16 H=32 Hkv=8."""
     import torch
 
     import exact_io_aware_94_b200 as fa
@@ -534,6 +536,37 @@ def run_profile_case(args, device):
             for _ in range(calls):
                 fa.backward(q, k, v, o, g, lse, causal=True, ws=ws, stream=stream)
         nbytes = 0
+    elif args.profile_case == "varlen_small":
+        # 8 causal sequences of 512..4,096 tokens, H16 d128 (about 1 GB on the device)
+        lens = torch.randint(512, 4097, (8,), generator=torch.Generator().manual_seed(7)).to(torch.int32)
+        cu = torch.zeros(9, dtype=torch.int32)
+        cu[1:] = torch.cumsum(lens, 0)
+        tot, H, d = int(cu[-1]), 16, 128
+        q, k, v = (torch.randn(tot, H, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+        cu_d = cu.to(device)
+        for _ in range(calls):
+            fa.forward_varlen(q, k, v, cu_d, cu_d, int(lens.max()), causal=True, stream=stream)
+        nbytes = 0
+    elif args.profile_case == "decode_paged_small":
+        # paged, grouped heads: B16 H32 Hkv8 d128, 64-token pages, lengths U[1024, 8192]
+        B, H, Hkv, ps, nblk, d = 16, 32, 8, 64, 128, 128
+        cg = torch.Generator().manual_seed(6)
+        lens = torch.randint(1024, nblk * ps + 1, (B,), generator=cg).to(torch.int32)
+        used = [(int(n) + ps - 1) // ps for n in lens]
+        npg = sum(used)
+        perm = torch.randperm(npg, generator=cg).to(torch.int32)
+        table = torch.zeros(B, nblk, dtype=torch.int32)
+        at = 0
+        for b in range(B):
+            table[b, : used[b]] = perm[at:at + used[b]]
+            at += used[b]
+        kp, vp = (torch.randn(npg, Hkv, ps, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(2))
+        qd = torch.randn(B, H, d, generator=gen, device=device).to(torch.bfloat16)
+        ws = fa.workspace(fa.fa_decode_paged_workspace_size(B, H, nblk, ps, d), device)
+        t_d, l_d = table.to(device), lens.to(device)
+        for _ in range(calls):
+            fa.decode_paged(qd, kp, vp, t_d, l_d, ws=ws, stream=stream)
+        nbytes = int(lens.sum()) * Hkv * d * 2 * 2
     else:
         B, H, cap, d = 16, 32, 8192, 128
         kc, vc = (torch.randn(B, H, cap, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(2))
@@ -588,7 +621,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
-    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small"], default=None,
+    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small", "varlen_small", "decode_paged_small"],
+                    default=None,
                     help="run only this path W+K times for a profiler; no benchmark line")
     args = ap.parse_args(argv)
     if args.impl == "ours" and args.warmup < 3:
