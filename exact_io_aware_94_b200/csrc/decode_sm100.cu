@@ -22,13 +22,16 @@
 // "The general lesson" names paged attention among the ways of moving less
 // data).  A work item covers a group of query heads of one KV head, so every K
 // and V row it loads serves the whole group.
-//   fa_decode_paged_split  persistent CTAs over (b, kv head, head group, chunk).
+//   fa_decode_paged_tma    persistent CTAs over (b, kv head, head group, chunk); a
+//                          copy warp stages each 64-key slice of K and V into
+//                          shared memory with bulk copies, 8 warps compute.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
 
 #include "fa_internal.h"
+#include "ptx.cuh"
 
 namespace fa {
 namespace {
@@ -225,184 +228,266 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) fa_decode_split(DecodeParam
     }
 }
 
-// Paged cache, GG query heads per work item sharing one KV head.  Same lane
-// layout as fa_decode_split: D/8 lanes hold one key row; each lane keeps the
-// running statistics of all GG heads for its slice of keys.
-template <int D, int GG, int UNROLL, int MINB>
-__global__ void __launch_bounds__(kDecodeThreads, MINB) fa_decode_paged_split(DecodeParams p) {
-    constexpr int kLanesPerKey = D / 8;
-    constexpr int kGroupsPerWarp = 32 / kLanesPerKey;
-    constexpr int kGroups = (kDecodeThreads / 32) * kGroupsPerWarp;
-    constexpr int kStep = kGroups * UNROLL;
+// Paged decode with grouped heads, K/V staged through shared memory.  A work
+// item is (b, KV head, group of GG query heads, chunk): every K and V row it
+// reads serves the whole group.  Warp 8 copies each 64-key stage of the item
+// (page segments of K and V, valid rows only) with 1-D bulk copies into a ring
+// of kPgStages stages.  In warps 0-7, D/8 lanes hold one key row slice (8 bf16)
+// and keep, per head, a running max, a running sum and an 8-wide accumulator:
+// dot products and accumulation use packed FFMA2, and the accumulators are
+// rescaled only when a head's max grows by more than 2^8 (O = acc / l holds for
+// any common reference).  Bytes in flight are bounded by the ring (128 KB at
+// d = 128), not by registers.  Every wait is bounded; an abort drains the
+// copies in flight.
+constexpr int kPgStages = 4;
+constexpr int kPgStageKeys = 64;
+constexpr int kPgThreads = 288;  // 8 compute warps + 1 copy warp
 
-    __shared__ float red_m[GG][kGroups];
-    __shared__ float red_l[GG][kGroups];
-    __shared__ float red_acc[GG][kGroups][D];
-    __shared__ int s_item[4];
+template <int D, int GG>
+struct PagedTmaLayout {
+    static constexpr int kLanesPerKey = D / 8;
+    static constexpr int kGroups = 8 * (32 / kLanesPerKey);
+    static constexpr int kStageBytes = kPgStageKeys * D * 2;  // one of K or V
+    static constexpr int kKOff = 0;
+    static constexpr int kVOff = kKOff + kPgStages * kStageBytes;
+    static constexpr int kRedMOff = kVOff + kPgStages * kStageBytes;
+    static constexpr int kRedLOff = kRedMOff + GG * kGroups * 4;
+    static constexpr int kRedAccOff = kRedLOff + GG * kGroups * 4;
+    static constexpr int kBarOff = (kRedAccOff + GG * kGroups * D * 4 + 7) / 8 * 8;
+    static constexpr int kMiscOff = kBarOff + 2 * kPgStages * 8;
+    static constexpr int kBytes = kMiscOff + 16 + 128;
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+template <int D, int GG>
+__global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParams p) {
+    using Lay = PagedTmaLayout<D, GG>;
+    constexpr int kLanesPerKey = Lay::kLanesPerKey;
+    constexpr int kGroupsPerWarp = 32 / kLanesPerKey;
+    constexpr int kGroups = Lay::kGroups;
+    constexpr int kKeysPerGroup = kPgStageKeys / kGroups;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    __nv_bfloat16* sk = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kKOff);
+    __nv_bfloat16* sv = reinterpret_cast<__nv_bfloat16*>(smem + Lay::kVOff);
+    float* red_m = reinterpret_cast<float*>(smem + Lay::kRedMOff);    // [GG][kGroups]
+    float* red_l = reinterpret_cast<float*>(smem + Lay::kRedLOff);    // [GG][kGroups]
+    float* red_acc = reinterpret_cast<float*>(smem + Lay::kRedAccOff);  // [GG][kGroups][D]
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
+    uint64_t* empty = full + kPgStages;
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;
-    const int e0 = (lane % kLanesPerKey) * 8;
-    const float sl2 = p.scale_log2;
-    const int group = p.H / p.Hkv;      // query heads per KV head
-    const int n_hg = group / GG;        // head groups per KV head
-    const int per_chunk = p.Hkv * n_hg;  // items per chunk of a sequence
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kPgStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 8);
+        }
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int group = p.H / p.Hkv;
+    const int n_hg = group / GG;
+    const int per_chunk = p.Hkv * n_hg;
     const int total = p.cum[p.B] * per_chunk;
     const int ps_mask = (1 << p.page_shift) - 1;
-
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        if (threadIdx.x == 0) {
-            // item -> (b, kv head, chunk, head group), ordered by b, then kv head, then
-            // chunk, then head group: the head groups of one chunk run side by side, so
-            // all but the first find that chunk's K and V rows in L2.
-            int lo = 0, hi = p.B;
-            while (hi - lo > 1) {
-                const int mid = (lo + hi) >> 1;
-                if (p.cum[mid] * per_chunk <= item) lo = mid; else hi = mid;
-            }
-            const int nb = p.cum[lo + 1] - p.cum[lo];
-            const int local = item - p.cum[lo] * per_chunk;
-            const int rem = local % (nb * n_hg);
-            s_item[0] = lo;
-            s_item[1] = local / (nb * n_hg);  // kv head
-            s_item[2] = rem % n_hg;           // head group
-            s_item[3] = rem / n_hg;           // chunk
+    const float sl2 = p.scale_log2;
+    // item -> (b, kv head, head group, chunk); every warp decodes it the same way
+    auto decode_item = [&](int item, int& b, int& hkv, int& hg, int& chunk) {
+        int lo = 0, hi = p.B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.cum[mid] * per_chunk <= item) lo = mid; else hi = mid;
         }
-        __syncthreads();
-        const int b = s_item[0], hkv = s_item[1], hg = s_item[2], chunk = s_item[3];
-        const int h0 = hkv * group + hg * GG;  // first query head of this item
-        const int len = p.lens[b];
-        const int start = chunk * kDecodeSplit;
-        const int end = min(start + kDecodeSplit, len);
-        const int* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
-        const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.k) + e0;
-        const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.v) + e0;
+        const int nb = p.cum[lo + 1] - p.cum[lo];
+        const int local = item - p.cum[lo] * per_chunk;
+        const int rem = local % (nb * n_hg);
+        b = lo;
+        hkv = local / (nb * n_hg);
+        hg = rem % n_hg;
+        chunk = rem / n_hg;
+    };
 
-        // q as packed pairs (x = element 2i, y = element 2i+1) for FFMA2
-        float2 q2[GG][4];
-#pragma unroll
-        for (int gg = 0; gg < GG; ++gg) {
-            float qf[8];
-            unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                    (static_cast<size_t>(b) * p.H + h0 + gg) * D + e0),
-                    qf);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) q2[gg][i] = make_float2(qf[2 * i], qf[2 * i + 1]);
-        }
-        // Running statistics per head against a reference max m (deferred rescale:
-        // O = acc / l holds for any common reference, so acc and l are rescaled only
-        // when a head's max has grown by more than 2^8 in exp2 units).
-        float m[GG], l[GG];
-        float2 acc2[GG][4];
-#pragma unroll
-        for (int gg = 0; gg < GG; ++gg) {
-            m[gg] = -INFINITY;
-            l[gg] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc2[gg][i] = make_float2(0.0f, 0.0f);
-        }
-
-        for (int base = start; base < end; base += kStep) {
-            uint4 kr[UNROLL], vr[UNROLL];
-            bool valid[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int key = base + u * kGroups + g;
-                valid[u] = key < end;
-                int pg = valid[u] ? table[key >> p.page_shift] : 0;
-                pg = (static_cast<unsigned>(pg) < static_cast<unsigned>(p.num_pages)) ? pg : 0;  // flagged by the plan
-                const size_t row = (static_cast<size_t>(pg) * p.Hkv + hkv) * (ps_mask + 1) + (key & ps_mask);
-                kr[u] = valid[u] ? ld_stream_u4(kbase + row * D) : make_uint4(0, 0, 0, 0);
-                vr[u] = valid[u] ? ld_stream_u4(vbase + row * D) : make_uint4(0, 0, 0, 0);
-            }
-            float s[UNROLL][GG];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const float2 k2[4] = {make_float2(__uint_as_float(kr[u].x << 16), __uint_as_float(kr[u].x & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(kr[u].y << 16), __uint_as_float(kr[u].y & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(kr[u].z << 16), __uint_as_float(kr[u].z & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(kr[u].w << 16), __uint_as_float(kr[u].w & 0xFFFF0000u))};
-#pragma unroll
-                for (int gg = 0; gg < GG; ++gg) {
-                    float2 d2 = __fmul2_rn(q2[gg][0], k2[0]);
-#pragma unroll
-                    for (int i = 1; i < 4; ++i) d2 = __ffma2_rn(q2[gg][i], k2[i], d2);
-                    float dot = d2.x + d2.y;
-#pragma unroll
-                    for (int o = kLanesPerKey / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-                    s[u][gg] = valid[u] ? dot : -INFINITY;
+    if (warp == 8) {
+        // ---------------- copy warp
+        int st = 0;  // stages issued
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
+            int b, hkv, hg, chunk;
+            decode_item(item, b, hkv, hg, chunk);
+            const int start = chunk * kDecodeSplit;
+            const int end = min(start + kDecodeSplit, p.lens[b]);
+            const int* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+            for (int k0 = start; k0 < end; k0 += kPgStageKeys, ++st) {
+                const int s = st % kPgStages;
+                if (st >= kPgStages) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / kPgStages) - 1) & 1, abort_flag, p.status));
+                    if (!ok) break;
                 }
+                const int n = min(kPgStageKeys, end - k0);
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(n) * D * 2 * 2);
+                    for (int key = k0; key < k0 + n;) {
+                        int pg = table[key >> p.page_shift];
+                        pg = (static_cast<unsigned>(pg) < static_cast<unsigned>(p.num_pages)) ? pg : 0;  // flagged by the plan
+                        const int r0 = key & ps_mask;
+                        const int seg = min(ps_mask + 1 - r0, k0 + n - key);
+                        const size_t row = (static_cast<size_t>(pg) * p.Hkv + hkv) * (ps_mask + 1) + r0;
+                        bulk_load(sk + (static_cast<size_t>(s) * kPgStageKeys + (key - k0)) * D,
+                                  static_cast<const __nv_bfloat16*>(p.k) + row * D, static_cast<uint32_t>(seg) * D * 2,
+                                  &full[s]);
+                        bulk_load(sv + (static_cast<size_t>(s) * kPgStageKeys + (key - k0)) * D,
+                                  static_cast<const __nv_bfloat16*>(p.v) + row * D, static_cast<uint32_t>(seg) * D * 2,
+                                  &full[s]);
+                        key += seg;
+                    }
+                }
+                __syncwarp();
             }
-            bool grow = false;
-            float mb[GG];
+        }
+        if (*abort_flag) {
+            // copies already issued land before the CTA's shared memory goes away
+            for (int t = max(0, st - kPgStages); t < st; ++t) mbar_wait_drain(&full[t % kPgStages], (t / kPgStages) & 1, p.status);
+        }
+    } else {
+        // ---------------- compute warps 0-7
+        const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;
+        const int e0 = (lane % kLanesPerKey) * 8;
+        int st = 0;  // stages consumed
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
+            int b, hkv, hg, chunk;
+            decode_item(item, b, hkv, hg, chunk);
+            const int h0 = hkv * group + hg * GG;
+            const int start = chunk * kDecodeSplit;
+            const int end = min(start + kDecodeSplit, p.lens[b]);
+            float2 q2[GG][4];
 #pragma unroll
             for (int gg = 0; gg < GG; ++gg) {
-                mb[gg] = s[0][gg];
+                float qf[8];
+                unpack8(*reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
+                                                        (static_cast<size_t>(b) * p.H + h0 + gg) * D + e0),
+                        qf);
 #pragma unroll
-                for (int u = 1; u < UNROLL; ++u) mb[gg] = fmaxf(mb[gg], s[u][gg]);
-                grow |= (m[gg] == -INFINITY) ? (mb[gg] != -INFINITY) : ((mb[gg] - m[gg]) * sl2 > 8.0f);
+                for (int i = 0; i < 4; ++i) q2[gg][i] = make_float2(qf[2 * i], qf[2 * i + 1]);
             }
-            if (__any_sync(0xffffffffu, grow)) {  // warp-uniform, rare after the first keys
+            float m[GG], l[GG];
+            float2 acc2[GG][4];
+#pragma unroll
+            for (int gg = 0; gg < GG; ++gg) {
+                m[gg] = -INFINITY;
+                l[gg] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc2[gg][i] = make_float2(0.0f, 0.0f);
+            }
+            for (int k0 = start; k0 < end; k0 += kPgStageKeys, ++st) {
+                const int s = st % kPgStages;
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (st / kPgStages) & 1, abort_flag, p.status));
+                if (!ok) break;
+                const int n = min(kPgStageKeys, end - k0);
+                float sc[kKeysPerGroup][GG];
+                uint4 vr[kKeysPerGroup];
+#pragma unroll
+                for (int u = 0; u < kKeysPerGroup; ++u) {
+                    const int kl = u * kGroups + g;
+                    const bool valid = kl < n;
+                    const size_t off = (static_cast<size_t>(s) * kPgStageKeys + kl) * D + e0;
+                    const uint4 kr = valid ? *reinterpret_cast<const uint4*>(sk + off) : make_uint4(0, 0, 0, 0);
+                    vr[u] = valid ? *reinterpret_cast<const uint4*>(sv + off) : make_uint4(0, 0, 0, 0);
+                    const float2 k2[4] = {make_float2(__uint_as_float(kr.x << 16), __uint_as_float(kr.x & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(kr.y << 16), __uint_as_float(kr.y & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(kr.z << 16), __uint_as_float(kr.z & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(kr.w << 16), __uint_as_float(kr.w & 0xFFFF0000u))};
+#pragma unroll
+                    for (int gg = 0; gg < GG; ++gg) {
+                        float2 d2 = __fmul2_rn(q2[gg][0], k2[0]);
+#pragma unroll
+                        for (int i = 1; i < 4; ++i) d2 = __ffma2_rn(q2[gg][i], k2[i], d2);
+                        float dot = d2.x + d2.y;
+#pragma unroll
+                        for (int o = kLanesPerKey / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+                        sc[u][gg] = valid ? dot : -INFINITY;
+                    }
+                }
+                // the stage's rows are in registers: hand it back to the copy warp
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                bool grow = false;
+                float mb[GG];
 #pragma unroll
                 for (int gg = 0; gg < GG; ++gg) {
-                    const float m_new = fmaxf(m[gg], mb[gg]);
-                    const float alpha = (m[gg] == -INFINITY) ? 0.0f : ex2f_approx((m[gg] - m_new) * sl2);
-                    l[gg] *= alpha;
-                    const float2 a2 = make_float2(alpha, alpha);
+                    mb[gg] = sc[0][gg];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc2[gg][i] = __fmul2_rn(acc2[gg][i], a2);
-                    m[gg] = m_new;
+                    for (int u = 1; u < kKeysPerGroup; ++u) mb[gg] = fmaxf(mb[gg], sc[u][gg]);
+                    grow |= (m[gg] == -INFINITY) ? (mb[gg] != -INFINITY) : ((mb[gg] - m[gg]) * sl2 > 8.0f);
+                }
+                if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+                    for (int gg = 0; gg < GG; ++gg) {
+                        const float m_new = fmaxf(m[gg], mb[gg]);
+                        const float alpha = (m[gg] == -INFINITY) ? 0.0f : ex2f_approx((m[gg] - m_new) * sl2);
+                        l[gg] *= alpha;
+                        const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc2[gg][i] = __fmul2_rn(acc2[gg][i], a2);
+                        m[gg] = m_new;
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kKeysPerGroup; ++u) {
+                    const float2 v2[4] = {make_float2(__uint_as_float(vr[u].x << 16), __uint_as_float(vr[u].x & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(vr[u].y << 16), __uint_as_float(vr[u].y & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(vr[u].z << 16), __uint_as_float(vr[u].z & 0xFFFF0000u)),
+                                          make_float2(__uint_as_float(vr[u].w << 16), __uint_as_float(vr[u].w & 0xFFFF0000u))};
+#pragma unroll
+                    for (int gg = 0; gg < GG; ++gg) {
+                        const float mbias = (m[gg] == -INFINITY) ? 0.0f : m[gg] * sl2;
+                        const float pu = ex2f_approx(fmaf(sc[u][gg], sl2, -mbias));
+                        l[gg] += pu;
+                        const float2 p2 = make_float2(pu, pu);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc2[gg][i] = __ffma2_rn(p2, v2[i], acc2[gg][i]);
+                    }
                 }
             }
+            if (!ok) break;
+            // merge the key groups of the 8 compute warps, per head
 #pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const float2 v2[4] = {make_float2(__uint_as_float(vr[u].x << 16), __uint_as_float(vr[u].x & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(vr[u].y << 16), __uint_as_float(vr[u].y & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(vr[u].z << 16), __uint_as_float(vr[u].z & 0xFFFF0000u)),
-                                      make_float2(__uint_as_float(vr[u].w << 16), __uint_as_float(vr[u].w & 0xFFFF0000u))};
+            for (int gg = 0; gg < GG; ++gg) {
+                if (lane % kLanesPerKey == 0) {
+                    red_m[gg * kGroups + g] = m[gg];
+                    red_l[gg * kGroups + g] = l[gg];
+                }
 #pragma unroll
-                for (int gg = 0; gg < GG; ++gg) {
-                    // m = -inf only while no valid key was seen: then every p is 0
-                    const float mbias = (m[gg] == -INFINITY) ? 0.0f : m[gg] * sl2;
-                    const float pu = ex2f_approx(fmaf(s[u][gg], sl2, -mbias));  // 0 for invalid keys
-                    l[gg] += pu;
-                    const float2 p2 = make_float2(pu, pu);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) acc2[gg][i] = __ffma2_rn(p2, v2[i], acc2[gg][i]);
+                for (int i = 0; i < 4; ++i) {
+                    red_acc[(gg * kGroups + g) * D + e0 + 2 * i] = acc2[gg][i].x;
+                    red_acc[(gg * kGroups + g) * D + e0 + 2 * i + 1] = acc2[gg][i].y;
                 }
             }
-        }
-
-        // merge the key groups of this CTA, per head
-#pragma unroll
-        for (int gg = 0; gg < GG; ++gg) {
-            if (lane % kLanesPerKey == 0) {
-                red_m[gg][g] = m[gg];
-                red_l[gg][g] = l[gg];
+            named_bar_sync(1, 256);
+            for (int t = threadIdx.x; t < GG * D; t += 256) {
+                const int gg = t / D, c = t % D;
+                float M = -INFINITY;
+                for (int i = 0; i < kGroups; ++i) M = fmaxf(M, red_m[gg * kGroups + i]);
+                float L = 0.0f, O = 0.0f;
+                for (int i = 0; i < kGroups; ++i) {
+                    const float mi = red_m[gg * kGroups + i];
+                    if (mi == -INFINITY) continue;
+                    const float w = ex2f_approx((mi - M) * sl2);
+                    L = fmaf(w, red_l[gg * kGroups + i], L);
+                    O = fmaf(w, red_acc[(gg * kGroups + i) * D + c], O);
+                }
+                const size_t slot = (static_cast<size_t>(b) * p.H + h0 + gg) * p.max_splits + chunk;
+                p.part_o[slot * D + c] = O / L;
+                if (c == 0) p.part_lse[slot] = M * p.scale + logf(L);
             }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                red_acc[gg][g][e0 + 2 * i] = acc2[gg][i].x;
-                red_acc[gg][g][e0 + 2 * i + 1] = acc2[gg][i].y;
-            }
+            named_bar_sync(1, 256);
         }
-        __syncthreads();
-        for (int t = threadIdx.x; t < GG * D; t += kDecodeThreads) {
-            const int gg = t / D, c = t % D;
-            float M = -INFINITY;
-            for (int i = 0; i < kGroups; ++i) M = fmaxf(M, red_m[gg][i]);
-            float L = 0.0f, O = 0.0f;
-            for (int i = 0; i < kGroups; ++i) {
-                if (red_m[gg][i] == -INFINITY) continue;
-                const float w = ex2f_approx((red_m[gg][i] - M) * sl2);
-                L = fmaf(w, red_l[gg][i], L);
-                O = fmaf(w, red_acc[gg][i][c], O);
-            }
-            const size_t slot = (static_cast<size_t>(b) * p.H + h0 + gg) * p.max_splits + chunk;
-            p.part_o[slot * D + c] = O / L;
-            if (c == 0) p.part_lse[slot] = M * p.scale + logf(L);
-        }
-        __syncthreads();
     }
 }
 
@@ -435,34 +520,25 @@ __global__ void __launch_bounds__(D) fa_decode_combine(DecodeParams p) {
     if (c == 0) p.lse[bh] = M + logf(L);
 }
 
-template <int D, int GG, int UNROLL, int MINB>
-cudaError_t launch_paged_split(const DecodeParams& p, int num_sms, cudaStream_t stream) {
+template <int D, int GG>
+cudaError_t launch_paged_tma(const DecodeParams& p, int num_sms, cudaStream_t stream) {
     const int n_hg = (p.H / p.Hkv) / GG;
     const long long upper = static_cast<long long>(p.B) * p.Hkv * n_hg * p.max_splits;
-    const int grid = static_cast<int>(std::min<long long>(upper, static_cast<long long>(num_sms) * MINB));
-    fa_decode_paged_split<D, GG, UNROLL, MINB><<<grid, kDecodeThreads, 0, stream>>>(p);
+    const int grid = static_cast<int>(std::min<long long>(upper, num_sms));
+    const int smem = PagedTmaLayout<D, GG>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(fa_decode_paged_tma<D, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fa_decode_paged_tma<D, GG><<<grid, kPgThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
-// Head-group width and, for groups of 4, unroll depth and CTAs per SM.  Groups of
-// 4 measured fastest (smaller groups re-read K/V through L2); 3 keys in flight per
-// lane group at 2 CTAs per SM beat 2 keys, and 4 keys at 1 CTA per SM.
-#ifndef FA_PAGED_GG
-#define FA_PAGED_GG 4
-#endif
-#ifndef FA_PG4_U
-#define FA_PG4_U 3
-#endif
-#ifndef FA_PG4_M
-#define FA_PG4_M 2
-#endif
 template <int D>
 cudaError_t launch_paged_d(const DecodeParams& p, int num_sms, cudaStream_t stream) {
     const int group = p.H / p.Hkv;
     cudaError_t e;
-    if (FA_PAGED_GG >= 4 && group % 4 == 0) e = launch_paged_split<D, 4, FA_PG4_U, FA_PG4_M>(p, num_sms, stream);
-    else if (FA_PAGED_GG >= 2 && group % 2 == 0) e = launch_paged_split<D, 2, 4, 2>(p, num_sms, stream);
-    else e = launch_paged_split<D, 1, 4, 3>(p, num_sms, stream);
+    if (group % 4 == 0) e = launch_paged_tma<D, 4>(p, num_sms, stream);
+    else if (group % 2 == 0) e = launch_paged_tma<D, 2>(p, num_sms, stream);
+    else e = launch_paged_tma<D, 1>(p, num_sms, stream);
     if (e != cudaSuccess) return e;
     fa_decode_combine<D><<<p.B * p.H, D, 0, stream>>>(p);
     return cudaGetLastError();
