@@ -67,6 +67,8 @@ def _load():
         lib.oracle_decode_paged.argtypes = [vp, vp, vp, c_int, vp, vp, dp, dp, i64, i64, i64, i64, i64, i64, i64,
                                             ctypes.c_double]
         lib.oracle_merge.restype = None
+        lib.oracle_forward_blocksparse.argtypes = [vp, vp, vp, c_int, dp, dp, vp, i64, i64, i64, i64, i64, i64,
+                                                   i64, i64, i64, ctypes.c_double, c_int]
         lib.oracle_merge.argtypes = [dp, dp, i64, i64, dp, dp]
         lib.oracle_num_threads.restype = c_int
         lib.oracle_num_threads.argtypes = []
@@ -213,6 +215,32 @@ def forward_varlen(q, k, v, cu_q, cu_k, scale: float, causal: bool):
     lse = np.empty((H, total_q), np.float64)
     _load().oracle_forward_varlen(pq, pk, pv, dt, o.ctypes.data, lse.ctypes.data, cq_.ctypes.data, ck_.ctypes.data,
                                   B, H, total_q, d, float(scale), int(bool(causal)))
+    return o, lse
+
+
+def forward_blocksparse(q, k, v, mask, scale: float, causal: bool, block_q: int = 128, block_k: int = 128):
+    """Forward under a block mask: q [B,H,Lq,d], k/v [B,H,Lk,d]; mask is uint8/bool, shape
+    [Tq, Tk], [H, Tq, Tk] or [B, H, Tq, Tk] with Tq = ceil(Lq/block_q), Tk = ceil(Lk/block_k)
+    (missing leading dimensions are shared).  Returns O [B,H,Lq,d] and LSE [B,H,Lq] in float64."""
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    if block_q < 1 or block_k < 1:
+        raise ValueError("block sizes must be >= 1")
+    tq, tk = -(-Lq // block_q), -(-Lk // block_k)
+    m = np.ascontiguousarray(np.asarray(mask).astype(np.uint8))
+    if m.shape[-2:] != (tq, tk) or m.ndim < 2 or m.ndim > 4 or (m.ndim >= 3 and m.shape[-3] != H) \
+            or (m.ndim == 4 and m.shape[0] != B):
+        raise ValueError("mask must have shape [Tq, Tk], [H, Tq, Tk] or [B, H, Tq, Tk]")
+    sb = tq * tk * H if m.ndim == 4 else 0
+    sh = tq * tk if m.ndim >= 3 else 0
+    kq, pq, cq = _as_input(q)
+    kk, pk, ck = _as_input(k)
+    kv, pv, cv = _as_input(v)
+    dt = _same_kind(cq, ck, cv)
+    o = np.empty((B, H, Lq, d), np.float64)
+    lse = np.empty((B, H, Lq), np.float64)
+    _load().oracle_forward_blocksparse(pq, pk, pv, dt, o.ctypes.data, lse.ctypes.data, m.ctypes.data, sb, sh,
+                                       int(block_q), int(block_k), B, H, Lq, Lk, d, float(scale), int(bool(causal)))
     return o, lse
 
 

@@ -193,6 +193,69 @@ void oracle_forward_varlen(const void* q, const void* k, const void* v, int dtyp
 }
 
 /*
+ * Forward pass under a block-sparse mask.  [G] "Common misconceptions" names a
+ * block-sparse extension that changes which query/key pairs attend, as
+ * distinct from the dense exact calculation; the pages give no mask format.
+ * Reading: the score matrix of each (b, h) is cut into blocks of block_q query
+ * rows by block_k key columns, and a byte per block says whether its pairs may
+ * attend (nonzero) or not (zero).  A key j is permitted for query row i when
+ * it is permitted by the dense rules (length bound and, with causal set, the
+ * bottom-right causal mask) AND its block is nonzero; the result is then the
+ * exact softmax attention over the permitted keys, two passes per row as in
+ * attend_row.  The mask of (b, h) starts at mask[b * mask_stride_b + h *
+ * mask_stride_h] and is row-major [ceil(Lq / block_q)][ceil(Lk / block_k)]
+ * (a stride of 0 shares one mask across that dimension).  A row with no
+ * permitted key has O = 0 and LSE = -inf.
+ */
+void oracle_forward_blocksparse(const void* q, const void* k, const void* v, int dtype, double* o,
+                                double* lse, const uint8_t* mask, int64_t mask_stride_b,
+                                int64_t mask_stride_h, int64_t block_q, int64_t block_k, int64_t B,
+                                int64_t H, int64_t Lq, int64_t Lk, int64_t d, double scale, int causal) {
+    const int64_t tk = (Lk + block_k - 1) / block_k;  /* key blocks per mask row */
+    const int64_t rows = B * H * Lq;
+#pragma omp parallel
+    {
+        double* t = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        int64_t* keys = (int64_t*)malloc(sizeof(int64_t) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < rows; ++r) {
+            const int64_t bh = r / Lq, i = r % Lq;
+            const int64_t b = bh / H, h = bh % H;
+            const uint8_t* mrow = mask + b * mask_stride_b + h * mask_stride_h + (i / block_q) * tk;
+            /* the permitted keys of row i, in increasing order */
+            const int64_t n_dense = oracle_permitted_keys(i, Lq, Lk, causal);
+            int64_t n = 0;
+            for (int64_t j = 0; j < n_dense; ++j)
+                if (mrow[j / block_k]) keys[n++] = j;
+            double* orow = o + r * d;
+            for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+            if (n == 0) {
+                lse[r] = -INFINITY;
+                continue;
+            }
+            const int64_t kv_off = bh * Lk * d;
+            double M = -INFINITY;
+            for (int64_t x = 0; x < n; ++x) {
+                double sdot = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    sdot += elem(q, r * d + c, dtype) * elem(k, kv_off + keys[x] * d + c, dtype);
+                t[x] = scale * sdot;
+                if (t[x] > M) M = t[x];
+            }
+            double Z = 0.0;
+            for (int64_t x = 0; x < n; ++x) Z += exp(t[x] - M);
+            for (int64_t x = 0; x < n; ++x) {
+                const double p = exp(t[x] - M) / Z;
+                for (int64_t c = 0; c < d; ++c) orow[c] += p * elem(v, kv_off + keys[x] * d + c, dtype);
+            }
+            lse[r] = M + log(Z);
+        }
+        free(keys);
+        free(t);
+    }
+}
+
+/*
  * Forward pass on a chosen set of rows.  rows[s] is a flat row index
  * (b*H + h)*Lq + i; the result for it goes to o_out[s*d ...] and lse_out[s].
  * Row sampling is exact: each row of the output depends on that query row

@@ -403,3 +403,101 @@ def test_varlen_forward_repacking_permutes_outputs():
         assert np.array_equal(lse2[:, cu2[new_b]:cu2[new_b + 1]], lse[:, cu[b]:cu[b + 1]])
     with pytest.raises(ValueError):
         oracle.forward_varlen(q, _pack(ks)[0], _pack(vs)[0], np.array([0, 5, 4, 11], np.int32), cu, 0.5, True)
+
+
+# ---- block-sparse forward: the dense rules AND a per-block mask over the score matrix.
+
+def _bs_inputs(seed, B, H, Lq, Lk, d):
+    g = torch.Generator("cpu").manual_seed(seed)
+    q = torch.randn(B, H, Lq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H, Lk, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, H, Lk, d, generator=g).to(torch.bfloat16)
+    return q, k, v
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("bq,bk", [(3, 5), (4, 4), (11, 1)])
+def test_blocksparse_all_ones_equals_dense(causal, bq, bk):
+    q, k, v = _bs_inputs(31, 2, 2, 11, 13, 6)
+    tq, tk = -(-11 // bq), -(-13 // bk)
+    o, lse = oracle.forward_blocksparse(q, k, v, np.ones((tq, tk), np.uint8), 0.4, causal, bq, bk)
+    od, ld = oracle.forward(q, k, v, 0.4, causal)
+    assert np.array_equal(o, od) and np.array_equal(lse, ld)
+
+
+def test_blocksparse_one_key_block_per_query_block():
+    """Query block r may see key block c(r) = (3r + 1) mod Tk only: its rows equal the dense
+    attention of those rows over that key block alone.  An asymmetric pattern, so reading
+    the mask transposed, or a block index off by one, fails."""
+    bq, bk, Lq, Lk = 4, 3, 14, 17
+    tq, tk = -(-Lq // bq), -(-Lk // bk)
+    q, k, v = _bs_inputs(32, 1, 2, Lq, Lk, 5)
+    mask = np.zeros((tq, tk), np.uint8)
+    cols = [(3 * r + 1) % tk for r in range(tq)]
+    for r, c in enumerate(cols):
+        mask[r, c] = 1
+    o, lse = oracle.forward_blocksparse(q, k, v, mask, 0.6, False, bq, bk)
+    for r, c in enumerate(cols):
+        rows = slice(r * bq, min(Lq, (r + 1) * bq))
+        keys = slice(c * bk, min(Lk, (c + 1) * bk))
+        od, ld = oracle.forward(q[:, :, rows].contiguous(), k[:, :, keys].contiguous(), v[:, :, keys].contiguous(),
+                                0.6, False)
+        assert np.max(np.abs(o[:, :, rows] - od)) <= 1e-12
+        assert np.max(np.abs(lse[:, :, rows] - ld)) <= 1e-12
+
+
+def test_blocksparse_complementary_masks_merge_to_dense():
+    """Splitting the key set of every row into two disjoint parts (a random block mask and its
+    complement) and merging the two results by their log-sum-exps gives the dense result:
+    the merge rule of the running statistics ([L] "The Three Running Statistics")."""
+    rng = np.random.default_rng(3)
+    bq, bk, Lq, Lk = 2, 3, 9, 10
+    tq, tk = -(-Lq // bq), -(-Lk // bk)
+    q, k, v = _bs_inputs(33, 2, 3, Lq, Lk, 4)
+    a = (rng.random((2, 3, tq, tk)) < 0.5).astype(np.uint8)
+    oa, la = oracle.forward_blocksparse(q, k, v, a, 0.5, False, bq, bk)
+    ob, lb = oracle.forward_blocksparse(q, k, v, 1 - a, 0.5, False, bq, bk)
+    od, ld = oracle.forward(q, k, v, 0.5, False)
+    lm = np.logaddexp(la, lb)
+    wa = np.where(np.isneginf(la), 0.0, np.exp(la - lm))[..., None]
+    wb = np.where(np.isneginf(lb), 0.0, np.exp(lb - lm))[..., None]
+    assert np.max(np.abs(lm - ld)) <= 1e-12
+    assert np.max(np.abs(wa * oa + wb * ob - od)) <= 1e-12
+
+
+def test_blocksparse_brute_force_per_head_masks_and_causal():
+    """Tiny case against an explicit element mask and a full softmax (brute force), with a
+    different mask per (b, h), a causal cut with Lq < Lk, and rows left with no key."""
+    rng = np.random.default_rng(4)
+    B, H, Lq, Lk, d, bq, bk, scale = 2, 2, 7, 10, 3, 2, 4, 0.7
+    tq, tk = -(-Lq // bq), -(-Lk // bk)
+    q, k, v = _bs_inputs(34, B, H, Lq, Lk, d)
+    mask = (rng.random((B, H, tq, tk)) < 0.5).astype(np.uint8)
+    mask[0, 1, 0, :] = 0  # rows 0-1 of (b=0, h=1) see nothing
+    o, lse = oracle.forward_blocksparse(q, k, v, mask, scale, True, bq, bk)
+    qd, kd, vd = (x.double().numpy() for x in (q, k, v))
+    for b in range(B):
+        for h in range(H):
+            for i in range(Lq):
+                allowed = [j for j in range(Lk) if j <= i + (Lk - Lq) and mask[b, h, i // bq, j // bk]]
+                if not allowed:
+                    assert np.all(o[b, h, i] == 0.0) and np.isneginf(lse[b, h, i])
+                    continue
+                t = np.array([scale * float(qd[b, h, i] @ kd[b, h, j]) for j in allowed])
+                w = np.exp(t - t.max())
+                ref = (w[:, None] * vd[b, h, allowed]).sum(0) / w.sum()
+                assert np.max(np.abs(o[b, h, i] - ref)) <= 1e-12
+                assert abs(lse[b, h, i] - (t.max() + np.log(w.sum()))) <= 1e-12
+    assert np.isneginf(lse[0, 1, :2]).all()
+
+
+def test_blocksparse_shared_mask_equals_replicated_and_checks_shape():
+    q, k, v = _bs_inputs(35, 2, 3, 8, 8, 4)
+    m = (np.random.default_rng(5).random((2, 2)) < 0.6).astype(np.uint8)
+    m[:, 0] = 1
+    o1, l1 = oracle.forward_blocksparse(q, k, v, m, 0.5, False, 4, 4)
+    o2, l2 = oracle.forward_blocksparse(q, k, v, np.broadcast_to(m, (3, 2, 2)), 0.5, False, 4, 4)
+    o3, l3 = oracle.forward_blocksparse(q, k, v, np.broadcast_to(m, (2, 3, 2, 2)), 0.5, False, 4, 4)
+    assert np.array_equal(o1, o2) and np.array_equal(o1, o3) and np.array_equal(l1, l3)
+    with pytest.raises(ValueError):
+        oracle.forward_blocksparse(q, k, v, np.ones((2, 3), np.uint8), 0.5, False, 4, 4)
