@@ -182,7 +182,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_INVALID_ARG;
     const long long n_ctas = static_cast<long long>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
@@ -226,7 +226,7 @@ int fa_decode(const void* q, const void* kcache, const void* vcache, const int* 
     if (!q || !kcache || !vcache || !kv_lens || !o || !lse) return FA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
-    if (!dims_ok(B, H, cap, d) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!dims_ok(B, H, cap, d) || !scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
         !aligned(kv_lens, 4) || !aligned(lse, 4))
         return FA_ERR_INVALID_ARG;
@@ -271,7 +271,7 @@ int fa_backward(const void* q, const void* k, const void* v, const void* o, cons
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
         !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
         return FA_ERR_INVALID_ARG;
@@ -319,7 +319,7 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
     if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (B <= 0 || H <= 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
         !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
         return FA_ERR_INVALID_ARG;
@@ -379,7 +379,7 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
     if (cap > 0x7FFFFFFFLL || static_cast<long long>(B) * H > (1LL << 30) ||
         static_cast<long long>(B) * max_blocks > 0x7FFFFFFFLL)
         return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kpages, 16) || !aligned(vpages, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
         !aligned(block_table, 4) || !aligned(kv_lens, 4))
         return FA_ERR_INVALID_ARG;

@@ -75,6 +75,10 @@ size_t bwd_workspace_bytes(int B, int H, int Lq);
 int prepare_device(int** status_ptr);
 int encode_tile_map(CUtensorMap* map, const void* base, int BH, int L, int d, int box_rows);
 bool shape_ok(int B, int H, int L, int d);
+// Every kernel takes the running maximum over raw scores q.k and applies the
+// scale inside the exponent, and masks scores to -inf before it: that is only
+// right for a positive, finite scale (zero would turn -inf * 0 into NaN).
+inline bool scale_ok(float scale) { return scale > 0.0f && scale <= 3.4028234663852886e38f; }
 cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream);
 
 // Decode: keys of each sequence are cut into chunks of kDecodeSplit keys.

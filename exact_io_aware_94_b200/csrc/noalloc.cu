@@ -53,7 +53,7 @@ extern "C" int fa_backward_noalloc(const void* q, const void* k, const void* v, 
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!shape_ok(B, H, Lq, d) || !shape_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-    if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq) ||
         !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
         return FA_ERR_INVALID_ARG;

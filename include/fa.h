@@ -28,6 +28,9 @@
  *               Causal calls require Lq <= Lk.
  *   LSE         LSE_i = ln sum_j exp(scale * q_i . k_j) over permitted keys
  *               (natural log, scaled-score units).
+ *   Scale       scale must be finite and > 0 (FA_ERR_INVALID_ARG otherwise): the
+ *               kernels take the running maximum over the raw scores q.k and
+ *               apply the scale inside the exponent.
  *   Pointers    All tensor pointers are DEVICE pointers on the current CUDA
  *               device, 16-byte aligned.  The caller owns every buffer; the
  *               library never allocates, frees or synchronises.  Calls are
@@ -51,7 +54,7 @@ extern "C" {
 
 typedef enum {
     FA_OK = 0,
-    FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, misalignment, causal with Lq > Lk */
+    FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size or scale, misalignment, causal with Lq > Lk */
     FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, dtype code unknown */
     FA_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than *_workspace_size() */
     FA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */

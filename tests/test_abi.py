@@ -66,6 +66,9 @@ P = 1 << 20
     (dict(q=P + 8), fa.FA_ERR_INVALID_ARG),
     (dict(o_dtype=7), fa.FA_ERR_UNSUPPORTED),
     (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),    # -inf masks times a zero scale would give NaN
+    (dict(scale=-0.125), fa.FA_ERR_INVALID_ARG),  # the running max is taken over raw scores
 ])
 def test_forward_argument_checks(lib, args, code):
     a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=1, Lq=64, Lk=64, d=64, scale=0.125, causal=0, o_dtype=0)
@@ -82,11 +85,13 @@ def test_forward_argument_checks(lib, args, code):
     (dict(ws=0), fa.FA_ERR_WORKSPACE),
     (dict(ws_bytes=16), fa.FA_ERR_WORKSPACE),
     (dict(ws=P + 16), fa.FA_ERR_WORKSPACE),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), fa.FA_ERR_INVALID_ARG),
 ])
 def test_decode_argument_checks(lib, args, code):
-    a = dict(q=P, k=P, v=P, kv=P, o=P, lse=P, B=2, H=2, cap=4096, d=128, ws=P, ws_bytes=1 << 30)
+    a = dict(q=P, k=P, v=P, kv=P, o=P, lse=P, B=2, H=2, cap=4096, d=128, ws=P, ws_bytes=1 << 30, scale=0.1)
     a.update(args)
-    rc = fa.fa_decode(a["q"], a["k"], a["v"], a["kv"], a["o"], a["lse"], a["B"], a["H"], a["cap"], a["d"], 0.1, 0,
+    rc = fa.fa_decode(a["q"], a["k"], a["v"], a["kv"], a["o"], a["lse"], a["B"], a["H"], a["cap"], a["d"], a["scale"], 0,
                       a["ws"], a["ws_bytes"], 0)
     assert rc == code
 
@@ -106,13 +111,14 @@ def test_decode_argument_checks(lib, args, code):
     (dict(ws=0), fa.FA_ERR_WORKSPACE),
     (dict(ws_bytes=16), fa.FA_ERR_WORKSPACE),
     (dict(ws=P + 16), fa.FA_ERR_WORKSPACE),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
 ])
 def test_decode_paged_argument_checks(lib, args, code):
     a = dict(q=P, kp=P, vp=P, bt=P, kv=P, o=P, lse=P, B=2, H=8, Hkv=2, pages=64, ps=16, blocks=32, d=128,
-             o_dtype=0, ws=P, ws_bytes=1 << 30)
+             o_dtype=0, ws=P, ws_bytes=1 << 30, scale=0.1)
     a.update(args)
     rc = fa.fa_decode_paged(a["q"], a["kp"], a["vp"], a["bt"], a["kv"], a["o"], a["lse"], a["B"], a["H"], a["Hkv"],
-                            a["pages"], a["ps"], a["blocks"], a["d"], 0.1, a["o_dtype"], a["ws"], a["ws_bytes"], 0)
+                            a["pages"], a["ps"], a["blocks"], a["d"], a["scale"], a["o_dtype"], a["ws"], a["ws_bytes"], 0)
     assert rc == code
 
 
@@ -133,13 +139,25 @@ def test_decode_paged_workspace_size(lib):
     (dict(o_dtype=3), fa.FA_ERR_UNSUPPORTED),
     (dict(tq=0), fa.FA_OK),            # nothing to do: no launch
     (dict(maxq=0), fa.FA_OK),
+    (dict(scale=-0.5), fa.FA_ERR_INVALID_ARG),
 ])
 def test_forward_varlen_argument_checks(lib, args, code):
-    a = dict(q=P, k=P, v=P, o=P, lse=P, cq=P, ck=P, B=3, H=4, tq=100, tk=120, maxq=64, d=128, o_dtype=0)
+    a = dict(q=P, k=P, v=P, o=P, lse=P, cq=P, ck=P, B=3, H=4, tq=100, tk=120, maxq=64, d=128, o_dtype=0, scale=0.1)
     a.update(args)
     rc = fa.fa_forward_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cq"], a["ck"], a["B"], a["H"], a["tq"],
-                              a["tk"], a["maxq"], a["d"], 0.1, 1, a["o_dtype"], 0)
+                              a["tk"], a["maxq"], a["d"], a["scale"], 1, a["o_dtype"], 0)
     assert rc == code
+
+
+@pytest.mark.parametrize("scale,code", [(0.125, fa.FA_ERR_WORKSPACE), (0.0, fa.FA_ERR_INVALID_ARG),
+                                        (-0.125, fa.FA_ERR_INVALID_ARG), (float("nan"), fa.FA_ERR_INVALID_ARG)])
+def test_backward_scale_checks(lib, scale, code):
+    """The backward masks scores to -inf before the exponent as the forward does: the
+    scale must be positive.  (A valid scale reaches the workspace check, which fails.)"""
+    rc = fa.fa_backward(P, P, P, P, P, P, P, P, P, 1, 1, 64, 64, 64, scale, 1, 0, 0, 0, 0)
+    assert rc == code
+    rc = fa.fa_backward_noalloc(P, P, P, P, P, P, P, P, P, 1, 1, 64, 64, 64, scale, 1, 0, 0)
+    assert rc == (fa.FA_ERR_INVALID_ARG if code == fa.FA_ERR_INVALID_ARG else rc)
 
 
 def test_decode_workspace_size(lib):
