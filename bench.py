@@ -351,7 +351,7 @@ def run_ours(args, dist, rank, world, device):
 
 
 def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
-    from exact_io_aware_94_b200.inputs import WORKLOADS
+    from exact_io_aware_94_b200.inputs import WORKLOADS, blocksparse_mask
 
     legs = {}
     steps = max(3, min(args.steps, 20))
@@ -462,6 +462,41 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                               "config": "16 causal sequences, lengths U[512, 8192] (%d tokens), H16 d128, packed"
                                         % tot}
     del qv, kv_, vv, ov, lv
+
+    # causal prefill under a block-sparse mask (sink + local window + 10% random blocks, per head)
+    w = WORKLOADS["prefill_blocksparse"]
+    Bs, Hs, Ls, ds = w["B"], w["H"], w["L"], w["d"]
+    mask = blocksparse_mask(Hs, Ls, Ls, seed=w["seed"], sink=w["sink"], window=w["window"], p_random=w["p_random"])
+    qs, ks, vs = (torch.randn(Bs, Hs, Ls, ds, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+    os_ = torch.empty(Bs, Hs, Ls, ds, dtype=torch.float32, device=device)
+    ls_ = torch.empty(Bs, Hs, Ls, dtype=torch.float32, device=device)
+    mask_d = mask.to(device)
+    tq = mask.shape[1]
+    wss = fa.workspace(fa.fa_forward_blocksparse_workspace_size(Bs, Hs, Ls, Ls), device)
+    sc_s = 1.0 / math.sqrt(ds)
+
+    def fwd_blocksparse():
+        rc = fa.fa_forward_blocksparse(qs, ks, vs, os_, ls_, mask_d, 0, tq * tq, Bs, Hs, Ls, Ls, ds, sc_s, 1,
+                                       fa.FA_DT_F32, wss, wss.numel(), stream)
+        assert rc == fa.FA_OK
+
+    # algorithmic work: 4 d FLOP per permitted (query, key) pair; with L a multiple of 128, a
+    # kept block below the diagonal holds 128 x 128 pairs and a diagonal block 128 x 129 / 2
+    r_ = torch.arange(tq)[:, None]
+    c_ = torch.arange(tq)[None, :]
+    pairs_blk = (c_ < r_).to(torch.float64) * 128 * 128 + (c_ == r_).to(torch.float64) * (128 * 129 // 2)
+    pairs = Bs * float((mask.to(torch.float64) * pairs_blk).sum())
+    fs = 4.0 * ds * pairs
+    density = pairs / (Bs * Hs * Ls * (Ls + 1) / 2)
+    t_s = time_steps(fwd_blocksparse, steps, warm, stream, dist, device) / steps
+    legs["prefill_blocksparse"] = {"ms": round(t_s * 1e3, 4), "TFLOP/s": round(fs / t_s / 1e12, 1),
+                                   "frac_of_peak": round(fs / t_s / 1e12 / peaks["bf16_tflops"], 4),
+                                   "launches": 2, "kernels": "fa_bsparse_plan + fa_fwd_kernel (block-sparse)",
+                                   "permitted_fraction_of_causal": round(density, 4),
+                                   "config": "B2 H16 L16384 d128 causal; per-head block mask: sink block, window "
+                                             "of 8 key blocks, 10% of other blocks below the diagonal; TFLOP/s "
+                                             "counts permitted pairs only"}
+    del qs, ks, vs, os_, ls_
 
     # paged cache with grouped heads: same batch and lengths, 8 KV heads for 32 query heads
     w = WORKLOADS["decode_paged_gqa"]

@@ -77,6 +77,11 @@ def load_library():
     lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, sz, vp]
     lib.fa_forward_varlen.restype = i
     lib.fa_forward_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, vp]
+    lib.fa_forward_blocksparse_workspace_size.restype = sz
+    lib.fa_forward_blocksparse_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_forward_blocksparse.restype = i
+    lib.fa_forward_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, i, i, i, i, i,
+                                           f, i, i, vp, sz, vp]
     lib.fa_decode_paged_workspace_size.restype = sz
     lib.fa_decode_paged_workspace_size.argtypes = [i, i, i, i, i]
     lib.fa_decode_paged.restype = i
@@ -150,6 +155,18 @@ def fa_forward_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q
     return load_library().fa_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
                                             _ptr(cu_seqlens_k), B, H, total_q, total_k, max_seqlen_q, d, float(scale),
                                             int(causal), int(o_dtype), _stream(stream))
+
+
+def fa_forward_blocksparse_workspace_size(B, H, Lq, Lk) -> int:
+    return int(load_library().fa_forward_blocksparse_workspace_size(B, H, Lq, Lk))
+
+
+def fa_forward_blocksparse(q, k, v, o, lse, block_mask, mask_stride_b, mask_stride_h, B, H, Lq, Lk, d, scale, causal,
+                           o_dtype, workspace, workspace_bytes, stream=None) -> int:
+    return load_library().fa_forward_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_mask),
+                                                 int(mask_stride_b), int(mask_stride_h), B, H, Lq, Lk, d,
+                                                 float(scale), int(causal), int(o_dtype), _ptr(workspace),
+                                                 int(workspace_bytes), _stream(stream))
 
 
 def fa_decode_paged_workspace_size(B, H, max_blocks, page_size, d) -> int:
@@ -286,4 +303,43 @@ def forward_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, scale=None
     rc = fa_forward_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, H, total_q, total_k, int(max_seqlen_q), d,
                            scale, causal, _DT[out_dtype], stream)
     _check(rc, "fa_forward_varlen")
+    return o, lse
+
+
+BLOCKSPARSE_BLOCK = 128
+
+
+def forward_blocksparse(q, k, v, block_mask, scale=None, causal=False, out_dtype=torch.float32, ws=None,
+                        stream=None):
+    """Forward under a block mask: bf16 q [B,H,Lq,d], k/v [B,H,Lk,d]; block_mask uint8 or bool on the device
+    with shape [Tq,Tk], [H,Tq,Tk] or [B,H,Tq,Tk] (Tq = ceil(Lq/128), Tk = ceil(Lk/128)); size-1 or
+    expanded leading dimensions are shared.  Returns O [B,H,Lq,d] (out_dtype) and LSE [B,H,Lq] (fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    B, H, Lq, d = q.shape
+    Lk = k.shape[2]
+    tq, tk = -(-Lq // BLOCKSPARSE_BLOCK), -(-Lk // BLOCKSPARSE_BLOCK)
+    m = block_mask
+    if not isinstance(m, torch.Tensor) or not m.is_cuda or m.dtype not in (torch.uint8, torch.bool):
+        raise ValueError("block_mask must be a CUDA uint8 or bool tensor")
+    if m.dtype == torch.bool:
+        m = m.view(torch.uint8)
+    while m.dim() < 4:
+        m = m.unsqueeze(0)
+    if m.dim() != 4 or tuple(m.shape[2:]) != (tq, tk) or m.shape[0] not in (1, B) or m.shape[1] not in (1, H) \
+            or m.stride(3) != 1 or (tq > 1 and m.stride(2) != tk):
+        raise ValueError("block_mask must have shape [Tq,Tk], [H,Tq,Tk] or [B,H,Tq,Tk] = [.., %d, %d] with "
+                         "contiguous rows" % (tq, tk))
+    sb = 0 if m.shape[0] == 1 else m.stride(0)
+    sh = 0 if m.shape[1] == 1 else m.stride(1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    nbytes = fa_forward_blocksparse_workspace_size(B, H, Lq, Lk)
+    if ws is None:
+        ws = workspace(nbytes, q.device)
+    o = torch.empty((B, H, Lq, d), dtype=out_dtype, device=q.device)
+    lse = torch.empty((B, H, Lq), dtype=torch.float32, device=q.device)
+    rc = fa_forward_blocksparse(q, k, v, o, lse, m, sb, sh, B, H, Lq, Lk, d, scale, causal, _DT[out_dtype], ws,
+                                ws.numel() * ws.element_size(), stream)
+    _check(rc, "fa_forward_blocksparse")
     return o, lse

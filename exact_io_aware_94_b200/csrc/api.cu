@@ -215,6 +215,76 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+size_t fa_forward_blocksparse_workspace_size(int B, int H, int Lq, int Lk) {
+    if (B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0) return 0;
+    if ((static_cast<long long>(Lk) + kFwdBN - 1) / kFwdBN > kBsMaxKeyBlocks) return 0;
+    return bs_workspace_bytes(B, H, Lq, Lk);
+}
+
+int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                           const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h, int B,
+                           int H, int Lq, int Lk, int d, float scale, int causal, int o_dtype, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
+    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+    if (mask_stride_b < 0 || mask_stride_h < 0) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+        return FA_ERR_INVALID_ARG;
+    const long long n_pairs = (Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    const long long tk = (static_cast<long long>(Lk) + kFwdBN - 1) / kFwdBN;
+    if (static_cast<long long>(B) * H * n_pairs > 0x7FFFFFFFLL || tk > kBsMaxKeyBlocks) return FA_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || workspace_bytes < bs_workspace_bytes(B, H, Lq, Lk))
+        return FA_ERR_WORKSPACE;
+
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+
+    const size_t n_units = static_cast<size_t>(B) * H * n_pairs;
+    BsPlanParams plan{};
+    plan.mask = block_mask;
+    plan.stride_b = mask_stride_b;
+    plan.stride_h = mask_stride_h;
+    plan.count = static_cast<int*>(workspace);
+    plan.list = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
+                                            ((n_units * sizeof(int) + 255) & ~static_cast<size_t>(255)));
+    plan.B = B;
+    plan.H = H;
+    plan.Lq = Lq;
+    plan.Lk = Lk;
+    plan.n_pairs = static_cast<int>(n_pairs);
+    plan.tk = static_cast<int>(tk);
+    plan.causal = causal ? 1 : 0;
+
+    FwdParams p{};
+    const int BH = B * H;
+    if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, kFwdBM)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    if ((rc = encode_out_map_impl(&p.tm_o, o, BH, Lq, d, o_dtype)) != FA_OK) return rc;
+    p.o = o;
+    p.lse = lse;
+    p.status = st->status_ptr;
+    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    p.bs_count = plan.count;
+    p.bs_list = plan.list;
+    p.bs_tk = plan.tk;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = plan.causal;
+    p.o_dtype = o_dtype;
+    cudaError_t e = launch_fwd_blocksparse(plan, p, d, st->num_sms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t fa_decode_workspace_size(int B, int H, int cap, int d) {
     if (B <= 0 || H <= 0 || cap <= 0 || (d != 64 && d != 128)) return 0;
     return decode_workspace_bytes(B, H, cap, d);

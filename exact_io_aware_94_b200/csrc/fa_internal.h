@@ -43,6 +43,13 @@ struct __align__(64) FwdParams {
     const int* cu_q;
     const int* cu_k;
     int max_pairs;
+    // block-sparse forward (fa_forward_blocksparse): unit (b*H + h, pair) of the batched
+    // unit space keeps bs_count[(b*H + h) * n_pairs + pair] entries at bs_list + that index
+    // * bs_tk.  An entry is a key-block index (bits 0-13), bit 14 set when the pair's first
+    // 128-row query block may see it and bit 15 for the second.  Null otherwise.
+    const int* bs_count;
+    const uint16_t* bs_list;
+    int bs_tk;
     int B, H, Lq, Lk;
     float scale;       // multiplies q.k
     float scale_log2;  // scale * log2(e)
@@ -111,9 +118,24 @@ void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, in
 cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 
+// Block-sparse planning: per 256-row unit, the key blocks (after the causal cut)
+// that either of its two 128-row query blocks may see, in increasing order.
+constexpr int kBsMaxKeyBlocks = 1 << 14;
+constexpr int kBsEntryTile = (1 << 14) - 1;
+struct BsPlanParams {
+    const uint8_t* mask;  // block mask of (b, h) at mask + b * stride_b + h * stride_h, [Tq][Tk]
+    long long stride_b, stride_h;
+    int* count;           // [B*H*n_pairs]
+    uint16_t* list;       // [B*H*n_pairs][Tk]
+    int B, H, Lq, Lk, n_pairs, tk, causal;
+};
+size_t bs_workspace_bytes(int B, int H, int Lq, int Lk);
+
 int fwd_smem_bytes(int d);
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
+cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p, int d, int num_sms,
+                                   cudaStream_t stream);
 int encode_packed_map(CUtensorMap* map, const void* base, int total, int H, int d, int box_rows, int elem_bytes,
                       bool swizzle_box64);
 int encode_out_map(CUtensorMap* map, void* base, int BH, int L, int d, int o_dtype);

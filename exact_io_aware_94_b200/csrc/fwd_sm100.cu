@@ -154,13 +154,40 @@ __device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u, bool f
     return r;
 }
 
-template <bool VARLEN>
+// Block-sparse: the batched unit order; both query blocks of a pair walk the same list of
+// key blocks (the union of what either may see, planned before the launch), and a query
+// block masks out the entries it may not see.  The plan keeps at least one entry.
+__device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u) {
+    const int BH = p.B * p.H;
+    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    Unit r;
+    const int pair = n_pairs - 1 - u / BH;
+    r.bh = u % BH;
+    r.i0 = pair * kFwdRowsPerCta;
+    const int cnt = p.bs_count[static_cast<size_t>(r.bh) * n_pairs + pair];
+    r.n_kv0 = cnt;
+    r.n_kv1 = (r.i0 + kFwdBM < p.Lq) ? cnt : 0;
+    r.q0 = 0;
+    r.k0 = 0;
+    r.lq = p.Lq;
+    r.lk = p.Lk;
+    return r;
+}
+
+// The planned list of a block-sparse unit.
+__device__ __forceinline__ const uint16_t* bsparse_list(const FwdParams& p, const Unit& un) {
+    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    return p.bs_list + (static_cast<size_t>(un.bh) * n_pairs + un.i0 / kFwdRowsPerCta) * p.bs_tk;
+}
+
+template <bool VARLEN, bool BSPARSE>
 __device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag) {
     if constexpr (VARLEN) return unit_of_varlen(p, u, flag);
+    else if constexpr (BSPARSE) return unit_of_bsparse(p, u);
     else return unit_of(p, u);
 }
 
-template <int D, bool VARLEN>
+template <int D, bool VARLEN, bool BSPARSE>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
     using Lay = FwdLayout<D>;
     constexpr int S = Lay::kStages;
@@ -263,7 +290,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     if (lane == 0) ticket = atomicAdd(p.sched, 1u);
                     u = static_cast<int>(min(__shfl_sync(0xffffffffu, ticket, 0), static_cast<unsigned>(n_units)));
                     if (u >= n_units) break;
-                    un = get_unit<VARLEN>(p, u, true);
+                    un = get_unit<VARLEN, BSPARSE>(p, u, true);
                     if (!VARLEN || un.n_kv0 > 0 || un.n_kv1 > 0) break;
                 }
                 if (lane == 0) {
@@ -289,10 +316,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     return true;
                 };
                 if (!(ok = load_q(0))) break;
+                const uint16_t* bs_list = nullptr;
+                if constexpr (BSPARSE) bs_list = bsparse_list(p, un);
                 for (int j = 0; j < n_max; ++j, ++kc) {
                     const int s = kc % S;
+                    int kvt = j;  // key block loaded as the unit's j-th tile
+                    if constexpr (BSPARSE) kvt = __ldg(bs_list + j) & kBsEntryTile;
                     if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
-                    const int ky = VARLEN ? un.bh % p.H : j * kFwdBN;
+                    const int ky = VARLEN ? un.bh % p.H : kvt * kFwdBN;
                     const int kz = VARLEN ? un.k0 + j * kFwdBN : un.bh;
                     mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
                     for (int b = 0; b < Lay::kBoxes; ++b)
@@ -362,7 +393,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
-                const Unit un = get_unit<VARLEN>(p, u, false);
+                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
@@ -448,7 +479,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit un = get_unit<VARLEN>(p, u, false);
+            const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
             const int n = (w == 0) ? un.n_kv0 : un.n_kv1;
             if (n == 0) continue;
             const int tile_first_row = un.i0 + w * kFwdBM;
@@ -459,7 +490,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             float m_ref = -INFINITY;  // running max of raw scores q.k (reference for P~)
             float l = 0.0f;           // running sum of the unrounded P~: gives the LSE
             float corr = 0.0f;        // sum over tiles of (bf16(P~_max) - P~_max): l + corr normalises O
+            const uint16_t* bs_list = nullptr;
+            if constexpr (BSPARSE) bs_list = bsparse_list(p, un);
             for (int j = 0; j < n; ++j, ++ts) {
+                int bs_entry = 0;  // issued before the wait, used after it
+                if constexpr (BSPARSE) bs_entry = __ldg(bs_list + j);
                 // warp-uniform outcome: the TMEM accesses below are warp-collective
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[w], ts & 1, abort_flag, p.status));
                 if (!ok) break;
@@ -475,13 +510,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     }
                     tmem_wait_ld();
                 }
-                const int kv0 = j * kFwdBN;
-                const bool need_mask =
-                    (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) || (kv0 + kFwdBN > un.lk);
+                int kv0 = j * kFwdBN;
+                bool mine = true;  // block-sparse: this query block may see the tile
+                if constexpr (BSPARSE) {
+                    kv0 = (bs_entry & kBsEntryTile) * kFwdBN;
+                    mine = (bs_entry >> (14 + w)) & 1;
+                }
+                const int lim = mine ? limit : kv0 - 1;  // a tile it may not see is masked whole
+                const bool need_mask = !mine || (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) ||
+                                       (kv0 + kFwdBN > un.lk);
                 if (need_mask) {
 #pragma unroll
                     for (int c = 0; c < kFwdBN; ++c)
-                        if (kv0 + c > limit) s[c] = -INFINITY;
+                        if (kv0 + c > lim) s[c] = -INFINITY;
                 }
                 // Row max: eight independent chains, then a tree.
                 float mx;
@@ -576,7 +617,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 // the 128-byte-swizzled layout of the O tensor map (16-byte pieces
                 // XOR row % 8: no bank conflicts), and one lane issues the tile store.
                 // Rows past Lq are clipped by the copy engine.
-                const float inv_l = 1.0f / (l + corr);
+                // (block-sparse: a row that may see no key has l = 0 and gets O = 0, LSE = -inf)
+                const float den = l + corr;
+                const float inv_l = (BSPARSE && !(den > 0.0f)) ? 0.0f : 1.0f / den;
                 uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
                 const bool f32 = p.o_dtype == FA_DT_F32;
                 const int n_chunks = f32 ? D / 32 : D / 64;
@@ -657,6 +700,59 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
 }
 
+// Block-sparse planning, one warp per 256-row unit (b*H + h, pair): the key blocks
+// that either 128-row query block of the pair may see -- under the causal cut and
+// the length bound, and with its mask byte set -- compacted in increasing order by
+// a ballot over 32 blocks at a time.  Each entry records which of the two query
+// blocks may see it.  A unit that may see nothing keeps one entry (key block 0,
+// seen by neither), so that its rows are still written (O = 0, LSE = -inf).
+constexpr int kBsPlanThreads = 256;
+
+__global__ void __launch_bounds__(kBsPlanThreads) fa_bsparse_plan(const BsPlanParams q) {
+    const long long unit = (static_cast<long long>(blockIdx.x) * kBsPlanThreads + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long n_units = static_cast<long long>(q.B) * q.H * q.n_pairs;
+    if (unit >= n_units) return;  // warp-uniform
+    const int bh = static_cast<int>(unit / q.n_pairs);
+    const int pair = static_cast<int>(unit % q.n_pairs);
+    const int b = bh / q.H, h = bh % q.H;
+    const int off = q.Lk - q.Lq;  // causal: query i sits at key position i + off
+    int n[2];  // key blocks within the causal cut and the length bound, per query block
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        const int first = pair * kFwdRowsPerCta + w * kFwdBM;
+        if (first >= q.Lq) {
+            n[w] = 0;
+        } else if (q.causal) {
+            const int last = min(first + kFwdBM - 1, q.Lq - 1);
+            n[w] = min(q.tk, (last + off) / kFwdBN + 1);
+        } else {
+            n[w] = q.tk;
+        }
+    }
+    // mask rows of the two query blocks (the second is only read when it exists: n[1] > 0)
+    const uint8_t* m0 = q.mask + b * q.stride_b + h * q.stride_h + static_cast<long long>(2 * pair) * q.tk;
+    const uint8_t* m1 = m0 + q.tk;
+    uint16_t* out = q.list + unit * q.tk;
+    int cnt = 0;
+    const int n_max = max(n[0], n[1]);
+    for (int base = 0; base < n_max; base += 32) {
+        const int t = base + lane;
+        const bool s0 = t < n[0] && m0[t] != 0;
+        const bool s1 = t < n[1] && m1[t] != 0;
+        const unsigned keep = __ballot_sync(0xffffffffu, s0 || s1);
+        if (s0 || s1)
+            out[cnt + __popc(keep & ((1u << lane) - 1u))] =
+                static_cast<uint16_t>(t | (s0 ? 1 << 14 : 0) | (s1 ? 1 << 15 : 0));
+        cnt += __popc(keep);
+    }
+    if (cnt == 0) {
+        if (lane == 0) out[0] = 0;
+        cnt = 1;
+    }
+    if (lane == 0) q.count[unit] = cnt;
+}
+
 // The setmaxnreg split only works if the block was launched with at least as
 // many registers as the split hands out; otherwise the increase would wait
 // forever.  Refuse to launch a build whose register count does not cover it.
@@ -674,7 +770,7 @@ cudaError_t check_register_split(K kernel) {
 
 int fwd_smem_bytes(int d) { return d == 128 ? FwdLayout<128>::kBytes : FwdLayout<64>::kBytes; }
 
-template <int D, bool VARLEN>
+template <int D, bool VARLEN, bool BSPARSE>
 cudaError_t launch_fwd_kernel(const FwdParams& p, int num_sms, cudaStream_t stream) {
     const long long pairs = VARLEN ? p.max_pairs : (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
     const long long units = static_cast<long long>(p.B) * p.H * pairs;
@@ -682,20 +778,40 @@ cudaError_t launch_fwd_kernel(const FwdParams& p, int num_sms, cudaStream_t stre
     const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
     const int smem = fwd_smem_bytes(D);
     cudaError_t e;
-    if ((e = check_register_split(fa_fwd_kernel<D, VARLEN>)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(fa_fwd_kernel<D, VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-        cudaSuccess)
-        return e;
-    fa_fwd_kernel<D, VARLEN><<<grid, kFwdThreads, smem, stream>>>(p);
+    if ((e = check_register_split(fa_fwd_kernel<D, VARLEN, BSPARSE>)) != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fa_fwd_kernel<D, VARLEN, BSPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fa_fwd_kernel<D, VARLEN, BSPARSE><<<grid, kFwdThreads, smem, stream>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
-    return d == 128 ? launch_fwd_kernel<128, false>(p, num_sms, stream) : launch_fwd_kernel<64, false>(p, num_sms, stream);
+    return d == 128 ? launch_fwd_kernel<128, false, false>(p, num_sms, stream)
+                    : launch_fwd_kernel<64, false, false>(p, num_sms, stream);
 }
 
 cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream) {
-    return d == 128 ? launch_fwd_kernel<128, true>(p, num_sms, stream) : launch_fwd_kernel<64, true>(p, num_sms, stream);
+    return d == 128 ? launch_fwd_kernel<128, true, false>(p, num_sms, stream)
+                    : launch_fwd_kernel<64, true, false>(p, num_sms, stream);
+}
+
+cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p, int d, int num_sms,
+                                   cudaStream_t stream) {
+    const long long n_units = static_cast<long long>(plan.B) * plan.H * plan.n_pairs;
+    if (n_units == 0) return cudaSuccess;
+    const long long blocks = (n_units * 32 + kBsPlanThreads - 1) / kBsPlanThreads;
+    fa_bsparse_plan<<<static_cast<unsigned>(blocks), kBsPlanThreads, 0, stream>>>(plan);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return d == 128 ? launch_fwd_kernel<128, false, true>(p, num_sms, stream)
+                    : launch_fwd_kernel<64, false, true>(p, num_sms, stream);
+}
+
+size_t bs_workspace_bytes(int B, int H, int Lq, int Lk) {
+    const size_t n_units = static_cast<size_t>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+    const size_t tk = (static_cast<size_t>(Lk) + kFwdBN - 1) / kFwdBN;
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return up(n_units * sizeof(int)) + up(n_units * tk * sizeof(uint16_t));
 }
 
 }  // namespace fa

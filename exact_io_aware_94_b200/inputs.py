@@ -131,6 +131,28 @@ def paged_decode_inputs(B: int, H: int, Hkv: int, page_size: int, max_blocks: in
     return PagedDecodeInputs(q, kp, vp, table, kv_lens)
 
 
+def blocksparse_mask(H: int, Lq: int, Lk: int, seed: int, sink: int = 1, window: int = 8, p_random: float = 0.1,
+                     causal: bool = True, block: int = 128) -> torch.Tensor:
+    """uint8 [H, Tq, Tk] block mask (Tq = ceil(Lq/block), Tk = ceil(Lk/block)) for query blocks of
+    ``block`` rows and key blocks of ``block`` keys: per head, the first ``sink`` key blocks, the
+    ``window`` key blocks ending at the block holding the query block's last permitted key
+    (bottom-right causal position; the last key block when not causal), and each other block up to
+    there with probability ``p_random`` (one ``torch.rand`` draw per block, generator seeded with
+    ``seed``)."""
+    tq, tk = -(-Lq // block), -(-Lk // block)
+    gen = torch.Generator("cpu").manual_seed(seed)
+    draw = torch.rand(H, tq, tk, generator=gen) < p_random
+    r = torch.arange(tq)[:, None]
+    c = torch.arange(tk)[None, :]
+    if causal:
+        last = (torch.clamp((r + 1) * block - 1, max=Lq - 1) + (Lk - Lq)) // block
+    else:
+        last = torch.full_like(r, tk - 1)
+    reach = c <= last
+    keep = (c < sink) | ((c > last - window) & reach) | (draw & reach)
+    return keep.to(torch.uint8)
+
+
 # The workloads the library is measured and checked on.  Shapes and value
 # distributions follow the pages' sizes: the 4,096-token example, a training
 # shape at 8,192, a 65,536-token context and a decode batch over a long cache.
@@ -140,10 +162,15 @@ WORKLOADS = {
     "train_L8192": dict(kind="fwdbwd", B=2, H=16, L=8192, d=128, causal=True, q_scale=1.0, seed=3),
     "long_L65536": dict(kind="fwd", B=1, H=8, L=65536, d=128, causal=True, q_scale=1.0, seed=4),
     "decode_cap32768": dict(kind="decode", B=64, H=32, cap=32768, d=128, len_lo=1024, len_hi=32768, seed=5),
-    # Paged cache with grouped heads: the same batch and lengths as the decode workload,
-    # 8 KV heads shared by groups of 4 query heads, 64-token pages in shuffled order.
     # Packed prefill batch of 16 causal sequences of 512 to 8,192 tokens.
     "prefill_varlen": dict(kind="varlen", B=16, H=16, d=128, len_lo=512, len_hi=8192, causal=True, seed=7),
+    # Causal prefill under a block-sparse mask (one mask per head, shared by the batch): an
+    # attention-sink block, a local window of 8 key blocks ending at the diagonal, and 10% of
+    # the other blocks below the diagonal at random.
+    "prefill_blocksparse": dict(kind="blocksparse", B=2, H=16, L=16384, d=128, causal=True, sink=1, window=8,
+                                p_random=0.1, seed=8),
+    # Paged cache with grouped heads: the same batch and lengths as the decode workload,
+    # 8 KV heads shared by groups of 4 query heads, 64-token pages in shuffled order.
     "decode_paged_gqa": dict(kind="decode_paged", B=64, H=32, Hkv=8, page_size=64, max_blocks=512, d=128,
                              len_lo=1024, len_hi=32768, seed=6),
 }

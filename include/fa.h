@@ -211,6 +211,37 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
                     void* stream);
 
 /*
+ * Forward pass under a block-sparse mask.  The glossary entry's "Common
+ * misconceptions" names a block-sparse extension that changes which query/key
+ * pairs attend, as distinct from the dense exact calculation; the pages give no
+ * mask format, so this is the plainest one: the score matrix of each (b, h) is
+ * cut into blocks of FA_BLOCKSPARSE_BLOCK query rows by FA_BLOCKSPARSE_BLOCK
+ * keys, and one byte per block permits its pairs (nonzero) or removes them
+ * (zero) before the softmax.  A key is permitted for a query row when fa_forward
+ * would permit it (length bound, causal mask) AND its block byte is nonzero;
+ * the result is the exact softmax attention over the permitted keys.  A row
+ * with no permitted key gets O = 0 and LSE = -inf.
+ *   q, k, v, o, lse, scale, causal, o_dtype: as fa_forward.
+ *   block_mask: DEVICE bytes; the mask of (b, h) is row-major [Tq][Tk] at
+ *   block_mask + b * mask_stride_b + h * mask_stride_h, with
+ *   Tq = ceil(Lq / 128), Tk = ceil(Lk / 128); strides are in bytes, >= 0
+ *   (0 shares one mask across that dimension).  Only bytes inside these
+ *   [Tq][Tk] masks are read.  Lk <= 128 * 16384.
+ *   workspace: caller-owned device scratch of at least
+ *   fa_forward_blocksparse_workspace_size() bytes, 256-byte aligned; it holds
+ *   the per-unit lists of key blocks that a small planning kernel builds
+ *   before the forward kernel (both launched on `stream`).
+ * Blocks whose byte is zero cost no tensor-core work unless the other
+ * 128-row query block that shares a 256-row work unit needs them.
+ */
+#define FA_BLOCKSPARSE_BLOCK 128
+size_t fa_forward_blocksparse_workspace_size(int B, int H, int Lq, int Lk);
+int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                           const unsigned char* block_mask, long long mask_stride_b, long long mask_stride_h, int B,
+                           int H, int Lq, int Lk, int d, float scale, int causal, int o_dtype, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, returns the current device's status word (FA_OK if no
  * kernel recorded a condition since the last call) and clears it.  Returns
  * FA_ERR_CUDA if the synchronisation itself fails.

@@ -160,6 +160,41 @@ def test_backward_scale_checks(lib, scale, code):
     assert rc == (fa.FA_ERR_INVALID_ARG if code == fa.FA_ERR_INVALID_ARG else rc)
 
 
+@pytest.mark.parametrize("args,code", [
+    (dict(mask=0), fa.FA_ERR_INVALID_ARG),
+    (dict(q=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(o_dtype=4), fa.FA_ERR_UNSUPPORTED),
+    (dict(sb=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(sh=-8), fa.FA_ERR_INVALID_ARG),
+    (dict(Lq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=1, Lq=600, Lk=520), fa.FA_ERR_INVALID_ARG),
+    (dict(Lk=128 * 16384 + 1), fa.FA_ERR_INVALID_ARG),  # key-block index must fit 14 bits
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(o=P + 8), fa.FA_ERR_INVALID_ARG),
+    (dict(ws=0), fa.FA_ERR_WORKSPACE),
+    (dict(ws=P + 16), fa.FA_ERR_WORKSPACE),
+    (dict(ws_bytes=256), fa.FA_ERR_WORKSPACE),
+])
+def test_forward_blocksparse_argument_checks(lib, args, code):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, mask=P + 3, sb=0, sh=40, B=2, H=3, Lq=300, Lk=520, d=128, scale=0.1,
+             causal=0, o_dtype=0, ws=P, ws_bytes=1 << 30)
+    a.update(args)
+    rc = fa.fa_forward_blocksparse(a["q"], a["k"], a["v"], a["o"], a["lse"], a["mask"], a["sb"], a["sh"], a["B"],
+                                   a["H"], a["Lq"], a["Lk"], a["d"], a["scale"], a["causal"], a["o_dtype"], a["ws"],
+                                   a["ws_bytes"], 0)
+    assert rc == code
+
+
+def test_forward_blocksparse_workspace_size(lib):
+    # per 256-row unit: a count (int32) and a list of up to Tk key blocks (uint16), each part 256-aligned
+    n_units, tk = 2 * 3 * 2, 5
+    want = -(-n_units * 4 // 256) * 256 + -(-n_units * tk * 2 // 256) * 256
+    assert fa.fa_forward_blocksparse_workspace_size(2, 3, 300, 520) == want
+    assert fa.fa_forward_blocksparse_workspace_size(0, 3, 300, 520) == 0
+    assert fa.fa_forward_blocksparse_workspace_size(1, 1, 128, 128 * 16384 + 1) == 0
+
+
 def test_decode_workspace_size(lib):
     # 2 heads x 4 chunks of 1024 keys x 128 fp32 + LSE + lengths + prefix sums
     n = fa.fa_decode_workspace_size(1, 2, 4096, 128)
