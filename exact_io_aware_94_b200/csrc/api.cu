@@ -249,9 +249,12 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
     plan.mask = block_mask;
     plan.stride_b = mask_stride_b;
     plan.stride_h = mask_stride_h;
-    plan.count = static_cast<int*>(workspace);
-    plan.list = reinterpret_cast<uint16_t*>(static_cast<char*>(workspace) +
-                                            ((n_units * sizeof(int) + 255) & ~static_cast<size_t>(255)));
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    char* ws = static_cast<char*>(workspace);
+    plan.meta = reinterpret_cast<int4*>(ws);
+    plan.list = reinterpret_cast<uint16_t*>(ws + up(n_units * sizeof(int4)));
+    plan.own = reinterpret_cast<uint16_t*>(ws + up(n_units * sizeof(int4)) +
+                                           up(n_units * static_cast<size_t>(tk) * sizeof(uint16_t)));
     plan.B = B;
     plan.H = H;
     plan.Lq = Lq;
@@ -270,8 +273,9 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
     p.lse = lse;
     p.status = st->status_ptr;
     p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
-    p.bs_count = plan.count;
+    p.bs_meta = plan.meta;
     p.bs_list = plan.list;
+    p.bs_own = plan.own;
     p.bs_tk = plan.tk;
     p.B = B;
     p.H = H;

@@ -43,12 +43,18 @@ struct __align__(64) FwdParams {
     const int* cu_q;
     const int* cu_k;
     int max_pairs;
-    // block-sparse forward (fa_forward_blocksparse): unit (b*H + h, pair) of the batched
-    // unit space keeps bs_count[(b*H + h) * n_pairs + pair] entries at bs_list + that index
-    // * bs_tk.  An entry is a key-block index (bits 0-13), bit 14 set when the pair's first
-    // 128-row query block may see it and bit 15 for the second.  Null otherwise.
-    const int* bs_count;
+    // block-sparse forward (fa_forward_blocksparse), per unit ui = (b*H + h) * n_pairs + pair:
+    //   bs_meta[ui] = {entries of the union list, union index of the last entry of query block 0,
+    //                  the same for query block 1 (-1 if it does not exist),
+    //                  own-list lengths n0 | n1 << 16};
+    //   union list at bs_list + ui * bs_tk: key-block index (bits 0-13), bit 14 / 15 set when
+    //   query block 0 / 1 of the pair takes part in the entry;
+    //   own list of query block w at bs_own + (2 * ui + w) * bs_tk: key-block index, bit 15
+    //   set when the block takes part only to write its empty rows (every score masked).
+    // Null otherwise.
+    const int4* bs_meta;
     const uint16_t* bs_list;
+    const uint16_t* bs_own;
     int bs_tk;
     int B, H, Lq, Lk;
     float scale;       // multiplies q.k
@@ -122,11 +128,13 @@ cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaS
 // that either of its two 128-row query blocks may see, in increasing order.
 constexpr int kBsMaxKeyBlocks = 1 << 14;
 constexpr int kBsEntryTile = (1 << 14) - 1;
+constexpr int kBsOwnMasked = 1 << 15;
 struct BsPlanParams {
     const uint8_t* mask;  // block mask of (b, h) at mask + b * stride_b + h * stride_h, [Tq][Tk]
     long long stride_b, stride_h;
-    int* count;           // [B*H*n_pairs]
+    int4* meta;           // [B*H*n_pairs]
     uint16_t* list;       // [B*H*n_pairs][Tk]
+    uint16_t* own;        // [B*H*n_pairs][2][Tk]
     int B, H, Lq, Lk, n_pairs, tk, causal;
 };
 size_t bs_workspace_bytes(int B, int H, int Lq, int Lk);

@@ -154,9 +154,14 @@ __device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u, bool f
     return r;
 }
 
-// Block-sparse: the batched unit order; both query blocks of a pair walk the same list of
-// key blocks (the union of what either may see, planned before the launch), and a query
-// block masks out the entries it may not see.  The plan keeps at least one entry.
+// Block-sparse: the batched unit order.  The producer and the MMA issuer walk the unit's
+// union list of key blocks (planned before the launch, at least one entry); each entry's
+// bits say which query block takes part in it.
+__device__ __forceinline__ size_t bsparse_index(const FwdParams& p, int bh, int i0) {
+    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    return static_cast<size_t>(bh) * n_pairs + i0 / kFwdRowsPerCta;
+}
+
 __device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
     const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
@@ -164,7 +169,7 @@ __device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u) {
     const int pair = n_pairs - 1 - u / BH;
     r.bh = u % BH;
     r.i0 = pair * kFwdRowsPerCta;
-    const int cnt = p.bs_count[static_cast<size_t>(r.bh) * n_pairs + pair];
+    const int cnt = p.bs_meta[bsparse_index(p, r.bh, r.i0)].x;
     r.n_kv0 = cnt;
     r.n_kv1 = (r.i0 + kFwdBM < p.Lq) ? cnt : 0;
     r.q0 = 0;
@@ -174,10 +179,9 @@ __device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u) {
     return r;
 }
 
-// The planned list of a block-sparse unit.
+// The planned union list of a block-sparse unit.
 __device__ __forceinline__ const uint16_t* bsparse_list(const FwdParams& p, const Unit& un) {
-    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
-    return p.bs_list + (static_cast<size_t>(un.bh) * n_pairs + un.i0 / kFwdRowsPerCta) * p.bs_tk;
+    return p.bs_list + bsparse_index(p, un.bh, un.i0) * p.bs_tk;
 }
 
 template <bool VARLEN, bool BSPARSE>
@@ -369,8 +373,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 }
                 umma_commit_w(&bar_s[w]);
             };
-            // PV for one half of the tile's keys (h = 0: keys 0-63, h = 1: keys 64-127).
-            auto issue_pv_half = [&](int w, int s, int j, int h) {
+            // PV for one half of the tile's keys (h = 0: keys 0-63, h = 1: keys 64-127);
+            // the warpgroup's first PV of a unit overwrites O_w.
+            auto issue_pv_half = [&](int w, int s, bool first, int h) {
                 const uint32_t t_p = tmem_base + w * 128;
                 const uint32_t t_o = tmem_base + 256 + w * D;
 #pragma unroll
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     const int kk = h * 4 + k4;
                     const uint64_t b =
                         smem_desc_sw128(sVa + s * Lay::kTileBytes + kk * 2048, Lay::kBoxBytes, 1024);
-                    umma_ts_w(t_o, t_p + kk * 8, b, kIdescPV, (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_ts_w(t_o, t_p + kk * 8, b, kIdescPV, (!first || kk > 0) ? 1u : 0u);
                 }
             };
             int kc = 0;                // K/V ring position
@@ -394,6 +399,84 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
                 const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
+                if constexpr (BSPARSE) {
+                    // Walk the union list; query block w takes part in entry j when bit 14 + w
+                    // is set.  Its S for an entry is issued one entry ahead, after its previous
+                    // PV (S_w and P_w share TMEM columns), its Q wait comes with its first S,
+                    // and its last S / PV release Q_w / hand O_w to the epilogue.
+                    const int4 meta = __ldg(p.bs_meta + bsparse_index(p, un.bh, un.i0));
+                    const uint16_t* lst = bsparse_list(p, un);
+                    const int n = meta.x;
+                    const int last[2] = {meta.y, meta.z};
+                    bool q_seen[2] = {false, false};
+                    bool pv_seen[2] = {false, false};
+                    int e_cur = __ldg(lst);
+                    int e_next = (n > 1) ? __ldg(lst + 1) : 0;
+                    if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int w = 0; w < 2; ++w) {
+                        if (!((e_cur >> (14 + w)) & 1)) continue;
+                        if (!(ok = wait(&bar_q[w], q_iter[w] & 1))) break;
+                        ++q_iter[w];
+                        q_seen[w] = true;
+                        tc_fence_after();
+                        issue_s(w, kc % S);
+                        if (last[w] == 0) umma_commit_w(&bar_q_free[w]);
+                    }
+                    if (!ok) break;
+                    umma_commit_w(&bar_kfree[kc % S]);
+                    for (int j = 0; ok && j < n; ++j) {
+                        const int e_after = (j + 2 < n) ? __ldg(lst + j + 2) : 0;  // in flight meanwhile
+                        const int s = (kc + j) % S;
+                        const int s1 = (kc + j + 1) % S;
+                        if (!(ok = wait(&bar_v[s], ((kc + j) / S) & 1))) break;
+                        bool k_ready = false;
+#pragma unroll
+                        for (int w = 0; w < 2; ++w) {
+                            if ((e_cur >> (14 + w)) & 1) {
+                                if (!pv_seen[w] && units_w[w] > 0) {
+                                    // O_w still holds the previous unit until its epilogue has read it
+                                    if (!(ok = wait(&bar_ofree[w], (units_w[w] - 1) & 1))) break;
+                                }
+                                if (!(ok = wait(&bar_p[2 * w], tp[w] & 1))) break;
+                                tc_fence_after();
+                                issue_pv_half(w, s, !pv_seen[w], 0);
+                                if (!(ok = wait(&bar_p[2 * w + 1], tp[w] & 1))) break;
+                                ++tp[w];
+                                tc_fence_after();
+                                issue_pv_half(w, s, !pv_seen[w], 1);
+                                pv_seen[w] = true;
+                                if (j == last[w]) {
+                                    umma_commit_w(&bar_o[w]);
+                                    ++units_w[w];
+                                }
+                            }
+                            if (j + 1 < n && ((e_next >> (14 + w)) & 1)) {
+                                if (!k_ready) {
+                                    if (!(ok = wait(&bar_k[s1], ((kc + j + 1) / S) & 1))) break;
+                                    tc_fence_after();
+                                    k_ready = true;
+                                }
+                                if (!q_seen[w]) {
+                                    if (!(ok = wait(&bar_q[w], q_iter[w] & 1))) break;
+                                    ++q_iter[w];
+                                    q_seen[w] = true;
+                                    tc_fence_after();
+                                }
+                                issue_s(w, s1);
+                                if (j + 1 == last[w]) umma_commit_w(&bar_q_free[w]);
+                            }
+                        }
+                        if (!ok) break;
+                        if (j + 1 < n) umma_commit_w(&bar_kfree[s1]);
+                        umma_commit_w(&bar_vfree[s]);
+                        e_cur = e_next;
+                        e_next = e_after;
+                    }
+                    kc += n;
+                    continue;
+                }
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
@@ -427,11 +510,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                             }
                             if (!(ok = wait(&bar_p[2 * w], tp[w] & 1))) break;
                             tc_fence_after();
-                            issue_pv_half(w, s, j, 0);
+                            issue_pv_half(w, s, j == 0, 0);
                             if (!(ok = wait(&bar_p[2 * w + 1], tp[w] & 1))) break;
                             ++tp[w];
                             tc_fence_after();
-                            issue_pv_half(w, s, j, 1);
+                            issue_pv_half(w, s, j == 0, 1);
                             if (j == nw - 1) {
                                 umma_commit_w(&bar_o[w]);
                                 ++units_w[w];
@@ -480,7 +563,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
             const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
-            const int n = (w == 0) ? un.n_kv0 : un.n_kv1;
+            int n = (w == 0) ? un.n_kv0 : un.n_kv1;
+            const uint16_t* bs_own = nullptr;  // block-sparse: this query block's own list
+            if constexpr (BSPARSE) {
+                const size_t ui = bsparse_index(p, un.bh, un.i0);
+                n = (__ldg(&p.bs_meta[ui].w) >> (16 * w)) & 0xffff;
+                bs_own = p.bs_own + (2 * ui + w) * p.bs_tk;
+            }
             if (n == 0) continue;
             const int tile_first_row = un.i0 + w * kFwdBM;
             const int row = tile_first_row + row_in_tile;
@@ -490,11 +579,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             float m_ref = -INFINITY;  // running max of raw scores q.k (reference for P~)
             float l = 0.0f;           // running sum of the unrounded P~: gives the LSE
             float corr = 0.0f;        // sum over tiles of (bf16(P~_max) - P~_max): l + corr normalises O
-            const uint16_t* bs_list = nullptr;
-            if constexpr (BSPARSE) bs_list = bsparse_list(p, un);
             for (int j = 0; j < n; ++j, ++ts) {
                 int bs_entry = 0;  // issued before the wait, used after it
-                if constexpr (BSPARSE) bs_entry = __ldg(bs_list + j);
+                if constexpr (BSPARSE) bs_entry = __ldg(bs_own + j);
                 // warp-uniform outcome: the TMEM accesses below are warp-collective
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[w], ts & 1, abort_flag, p.status));
                 if (!ok) break;
@@ -514,7 +601,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 bool mine = true;  // block-sparse: this query block may see the tile
                 if constexpr (BSPARSE) {
                     kv0 = (bs_entry & kBsEntryTile) * kFwdBN;
-                    mine = (bs_entry >> (14 + w)) & 1;
+                    mine = !(bs_entry & kBsOwnMasked);
                 }
                 const int lim = mine ? limit : kv0 - 1;  // a tile it may not see is masked whole
                 const bool need_mask = !mine || (p.causal && kv0 + kFwdBN - 1 > tile_first_row + off) ||
@@ -700,12 +787,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
 }
 
-// Block-sparse planning, one warp per 256-row unit (b*H + h, pair): the key blocks
-// that either 128-row query block of the pair may see -- under the causal cut and
-// the length bound, and with its mask byte set -- compacted in increasing order by
-// a ballot over 32 blocks at a time.  Each entry records which of the two query
-// blocks may see it.  A unit that may see nothing keeps one entry (key block 0,
-// seen by neither), so that its rows are still written (O = 0, LSE = -inf).
+// Block-sparse planning, one warp per 256-row unit (b*H + h, pair).  For each of the
+// unit's two 128-row query blocks, a key block is seen when it lies inside the causal
+// cut and the length bound and its mask byte is set.  Per 32 key blocks, one per lane,
+// ballots and popcounts compact, in increasing order:
+//   - the union list (key blocks either query block sees; bit 14 + w when block w does),
+//     which the producer loads and the MMA issuer walks;
+//   - each query block's own list, which its softmax warpgroup walks.
+// A query block that exists but sees nothing still takes part in one entry (the union's
+// first, or key block 0 when the union is empty), flagged kBsOwnMasked in its own list:
+// its scores are all masked, and its rows get O = 0 and LSE = -inf.
 constexpr int kBsPlanThreads = 256;
 
 __global__ void __launch_bounds__(kBsPlanThreads) fa_bsparse_plan(const BsPlanParams q) {
@@ -734,23 +825,49 @@ __global__ void __launch_bounds__(kBsPlanThreads) fa_bsparse_plan(const BsPlanPa
     const uint8_t* m0 = q.mask + b * q.stride_b + h * q.stride_h + static_cast<long long>(2 * pair) * q.tk;
     const uint8_t* m1 = m0 + q.tk;
     uint16_t* out = q.list + unit * q.tk;
-    int cnt = 0;
+    uint16_t* own0 = q.own + 2 * unit * q.tk;
+    uint16_t* own1 = own0 + q.tk;
+    const unsigned below = (1u << lane) - 1u;
+    int cnt = 0, c0 = 0, c1 = 0, last0 = -1, last1 = -1;
     const int n_max = max(n[0], n[1]);
     for (int base = 0; base < n_max; base += 32) {
         const int t = base + lane;
         const bool s0 = t < n[0] && m0[t] != 0;
         const bool s1 = t < n[1] && m1[t] != 0;
         const unsigned keep = __ballot_sync(0xffffffffu, s0 || s1);
-        if (s0 || s1)
-            out[cnt + __popc(keep & ((1u << lane) - 1u))] =
-                static_cast<uint16_t>(t | (s0 ? 1 << 14 : 0) | (s1 ? 1 << 15 : 0));
+        const unsigned k0 = __ballot_sync(0xffffffffu, s0);
+        const unsigned k1 = __ballot_sync(0xffffffffu, s1);
+        const int pos = cnt + __popc(keep & below);  // this lane's union index, if kept
+        if (s0 || s1) out[pos] = static_cast<uint16_t>(t | (s0 ? 1 << 14 : 0) | (s1 ? 1 << 15 : 0));
+        if (s0) own0[c0 + __popc(k0 & below)] = static_cast<uint16_t>(t);
+        if (s1) own1[c1 + __popc(k1 & below)] = static_cast<uint16_t>(t);
+        last0 = max(last0, __reduce_max_sync(0xffffffffu, s0 ? pos : -1));
+        last1 = max(last1, __reduce_max_sync(0xffffffffu, s1 ? pos : -1));
         cnt += __popc(keep);
+        c0 += __popc(k0);
+        c1 += __popc(k1);
     }
-    if (cnt == 0) {
-        if (lane == 0) out[0] = 0;
-        cnt = 1;
+    __syncwarp();  // the lists' writes are visible to lane 0 below
+    if (lane == 0) {
+        if (cnt == 0) {
+            out[0] = 0;
+            cnt = 1;
+        }
+        const int tile0 = out[0] & kBsEntryTile;
+        if (c0 == 0) {  // query block 0 always exists
+            out[0] = static_cast<uint16_t>(out[0] | (1 << 14));
+            own0[0] = static_cast<uint16_t>(tile0 | kBsOwnMasked);
+            c0 = 1;
+            last0 = max(last0, 0);
+        }
+        if (n[1] > 0 && c1 == 0) {
+            out[0] = static_cast<uint16_t>(out[0] | (1 << 15));
+            own1[0] = static_cast<uint16_t>(tile0 | kBsOwnMasked);
+            c1 = 1;
+            last1 = max(last1, 0);
+        }
+        q.meta[unit] = make_int4(cnt, last0, n[1] > 0 ? last1 : -1, c0 | (c1 << 16));
     }
-    if (lane == 0) q.count[unit] = cnt;
 }
 
 // The setmaxnreg split only works if the block was launched with at least as
@@ -811,7 +928,8 @@ size_t bs_workspace_bytes(int B, int H, int Lq, int Lk) {
     const size_t n_units = static_cast<size_t>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
     const size_t tk = (static_cast<size_t>(Lk) + kFwdBN - 1) / kFwdBN;
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    return up(n_units * sizeof(int)) + up(n_units * tk * sizeof(uint16_t));
+    // metadata, union lists, own lists (two per unit)
+    return up(n_units * sizeof(int4)) + up(n_units * tk * sizeof(uint16_t)) + up(2 * n_units * tk * sizeof(uint16_t));
 }
 
 }  // namespace fa

@@ -187,9 +187,11 @@ def test_forward_blocksparse_argument_checks(lib, args, code):
 
 
 def test_forward_blocksparse_workspace_size(lib):
-    # per 256-row unit: a count (int32) and a list of up to Tk key blocks (uint16), each part 256-aligned
+    # per 256-row unit: 16 bytes of metadata, a union list and two own lists of up to Tk key
+    # blocks (uint16 each); each of the three parts 256-byte aligned
     n_units, tk = 2 * 3 * 2, 5
-    want = -(-n_units * 4 // 256) * 256 + -(-n_units * tk * 2 // 256) * 256
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    want = up(n_units * 16) + up(n_units * tk * 2) + up(2 * n_units * tk * 2)
     assert fa.fa_forward_blocksparse_workspace_size(2, 3, 300, 520) == want
     assert fa.fa_forward_blocksparse_workspace_size(0, 3, 300, 520) == 0
     assert fa.fa_forward_blocksparse_workspace_size(1, 1, 128, 128 * 16384 + 1) == 0
