@@ -704,9 +704,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 // the 128-byte-swizzled layout of the O tensor map (16-byte pieces
                 // XOR row % 8: no bank conflicts), and one lane issues the tile store.
                 // Rows past Lq are clipped by the copy engine.
-                // (block-sparse: a row that may see no key has l = 0 and gets O = 0, LSE = -inf)
+                // Block-sparse: a row that may see no key has l = 0 and gets O = 0, LSE = -inf.
+                // Its accumulator is cleared rather than scaled: the fully masked tile it ran
+                // may hold non-finite V rows, and 0 * inf or 0 * NaN in the PV product is NaN.
                 const float den = l + corr;
                 const float inv_l = (BSPARSE && !(den > 0.0f)) ? 0.0f : 1.0f / den;
+                if constexpr (BSPARSE) {
+                    if (!(den > 0.0f)) {
+#pragma unroll
+                        for (int c = 0; c < D; ++c) ov[c] = 0u;
+                    }
+                }
                 uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
                 const bool f32 = p.o_dtype == FA_DT_F32;
                 const int n_chunks = f32 ? D / 32 : D / 64;

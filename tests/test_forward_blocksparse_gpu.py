@@ -39,8 +39,8 @@ def run_both(inp, mask_dev, mask_np, causal, dev, what):
 
 @pytest.mark.parametrize("causal", [True, False])
 def test_all_ones_mask_equals_dense_forward_bitwise(cuda_device, causal):
-    """With every block permitted the kernel does the dense forward's arithmetic in the same
-    order (a query block's extra, fully masked tile adds exact zeros): bit-identical output."""
+    """With every block permitted each query block walks the same key tiles as in the dense
+    forward, in the same order, with the same arithmetic: bit-identical output."""
     B, H, L, d = 1, 2, 700, 128
     inp = attention_inputs(B, H, L, L, d, seed=50)
     q, k, v = inp.q.to(cuda_device), inp.k.to(cuda_device), inp.v.to(cuda_device)
@@ -89,6 +89,29 @@ def test_rows_with_no_key_are_zero_with_lse_minus_inf(cuda_device):
     o, lse = fa.forward_blocksparse(inp.q.to(cuda_device), inp.k.to(cuda_device), inp.v.to(cuda_device),
                                     torch.from_numpy(mask).to(cuda_device), causal=True)
     assert (o[0, 1, 256:512] == 0).all() and torch.isneginf(lse[0, 1, 640:768]).all()
+
+
+def test_blocks_nobody_sees_hold_nan(cuda_device):
+    """K/V rows of key blocks that no query block may see are NaN.  A unit whose two query
+    blocks see nothing still runs one fully masked tile, which may be such a block: its rows
+    must still be exactly 0 with LSE = -inf, and every other row must match the oracle."""
+    B, H, L, d = 1, 2, 640, 128
+    inp = attention_inputs(B, H, L, L, d, seed=56)
+    t = tiles(L)
+    mask = np.zeros((H, t, t), np.uint8)
+    mask[:, 0:2, 4] = 1  # query blocks 0-1 see key block 4
+    mask[:, 4, 3] = 1    # query block 4 sees key block 3; blocks 2-3 (one unit) see nothing
+    k, v = inp.k.clone(), inp.v.clone()
+    k[:, :, : 3 * BLK] = float("nan")  # key blocks 0-2: seen by nobody
+    v[:, :, : 3 * BLK] = float("nan")
+    scale = 1.0 / math.sqrt(d)
+    o_ref, lse_ref = oracle.forward_blocksparse(inp.q, k, v, mask, scale, False, BLK, BLK)
+    o, lse = fa.forward_blocksparse(inp.q.to(cuda_device), k.to(cuda_device), v.to(cuda_device),
+                                    torch.from_numpy(mask).to(cuda_device), scale=scale)
+    assert fa.fa_check_status() == fa.FA_OK
+    assert (o[:, :, 2 * BLK:4 * BLK] == 0).all() and torch.isneginf(lse[:, :, 2 * BLK:4 * BLK]).all()
+    check_o(o, o_ref, "NaN in unseen blocks")
+    check_lse(lse, lse_ref, "NaN in unseen blocks")
 
 
 def test_shared_and_expanded_masks(cuda_device):
