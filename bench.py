@@ -48,6 +48,23 @@ def attn_flops(B, H, Lq, Lk, d, causal, backward=False):
     return f
 
 
+def blocksparse_pairs(mask, Lq, Lk, causal, block=128):
+    """Permitted (query, key) pairs under a block mask ([..., Tq, Tk], nonzero = permitted)
+    ANDed with the length bound and the bottom-right causal mask, summed over the mask's
+    leading dimensions: the algorithmic work of a block-sparse forward is 4 d FLOP per pair."""
+    import numpy as np
+
+    m = np.asarray(mask) != 0
+    tq, tk = m.shape[-2], m.shape[-1]
+    rows = np.arange(tq * block)[:, None]          # query row, padded to whole blocks
+    c0 = np.arange(tk)[None, :] * block             # first key of each key block
+    c1 = np.minimum(c0 + block, Lk)                 # one past its last key
+    hi = np.minimum(c1, rows + (Lk - Lq) + 1) if causal else np.broadcast_to(c1, (rows.shape[0], tk))
+    per_row = np.clip(hi - c0, 0, None) * (rows < Lq)  # [rows, tk] keys of each block per row
+    per_block = per_row.reshape(tq, block, tk).sum(1)  # [tq, tk]
+    return float((m * per_block).sum())
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -480,12 +497,8 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                        fa.FA_DT_F32, wss, wss.numel(), stream)
         assert rc == fa.FA_OK
 
-    # algorithmic work: 4 d FLOP per permitted (query, key) pair; with L a multiple of 128, a
-    # kept block below the diagonal holds 128 x 128 pairs and a diagonal block 128 x 129 / 2
-    r_ = torch.arange(tq)[:, None]
-    c_ = torch.arange(tq)[None, :]
-    pairs_blk = (c_ < r_).to(torch.float64) * 128 * 128 + (c_ == r_).to(torch.float64) * (128 * 129 // 2)
-    pairs = Bs * float((mask.to(torch.float64) * pairs_blk).sum())
+    # algorithmic work: 4 d FLOP per permitted (query, key) pair (the mask is shared by the batch)
+    pairs = Bs * blocksparse_pairs(mask.numpy(), Ls, Ls, True)
     fs = 4.0 * ds * pairs
     density = pairs / (Bs * Hs * Ls * (Ls + 1) / 2)
     t_s = time_steps(fwd_blocksparse, steps, warm, stream, dist, device) / steps
