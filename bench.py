@@ -561,7 +561,9 @@ def run_profile_case(args, device):
     bwd: forward then backward at the 8,192-token training shape; decode_small:
     decode at B=16 H=32 cap=8192 (1 GiB of cache, small enough to capture);
     varlen_small: packed causal forward of 8 sequences of 512..4,096 tokens;
-    decode_paged_small: paged, grouped-head decode at B=16 H=32 Hkv=8."""
+    decode_paged_small: paged, grouped-head decode at B=16 H=32 Hkv=8;
+    blocksparse_small: block-sparse causal forward at B=2 H=16 L=8192 with the
+    benchmark's mask recipe (192 MiB of Q/K/V, more than L2)."""
     import torch
 
     import exact_io_aware_94_b200 as fa
@@ -594,6 +596,18 @@ def run_profile_case(args, device):
         cu_d = cu.to(device)
         for _ in range(calls):
             fa.forward_varlen(q, k, v, cu_d, cu_d, int(lens.max()), causal=True, stream=stream)
+        nbytes = 0
+    elif args.profile_case == "blocksparse_small":
+        from exact_io_aware_94_b200.inputs import blocksparse_mask
+
+        w = WORKLOADS["prefill_blocksparse"]
+        B, H, L, d = 2, 16, 8192, 128
+        q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+        mask = blocksparse_mask(H, L, L, seed=w["seed"], sink=w["sink"], window=w["window"],
+                                p_random=w["p_random"]).to(device)
+        ws = fa.workspace(fa.fa_forward_blocksparse_workspace_size(B, H, L, L), device)
+        for _ in range(calls):
+            fa.forward_blocksparse(q, k, v, mask, causal=True, ws=ws, stream=stream)
         nbytes = 0
     elif args.profile_case == "decode_paged_small":
         # paged, grouped heads: B16 H32 Hkv8 d128, 64-token pages, lengths U[1024, 8192]
@@ -669,7 +683,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
-    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small", "varlen_small", "decode_paged_small"],
+    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small", "varlen_small", "decode_paged_small",
+                                                    "blocksparse_small"],
                     default=None,
                     help="run only this path W+K times for a profiler; no benchmark line")
     args = ap.parse_args(argv)
