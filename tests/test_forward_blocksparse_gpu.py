@@ -114,6 +114,20 @@ def test_blocks_nobody_sees_hold_nan(cuda_device):
     check_lse(lse, lse_ref, "NaN in unseen blocks")
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_all_zero_mask(cuda_device, causal):
+    """No block permitted anywhere: every unit runs only its one fully masked entry, and every
+    row gets O = 0 and LSE = -inf, in both output types."""
+    B, H, L, d = 2, 2, 333, 64
+    inp = attention_inputs(B, H, L, L, d, seed=57)
+    zeros = torch.zeros(tiles(L), tiles(L), dtype=torch.uint8, device=cuda_device)
+    for out_dtype in (torch.float32, torch.bfloat16):
+        o, lse = fa.forward_blocksparse(inp.q.to(cuda_device), inp.k.to(cuda_device), inp.v.to(cuda_device), zeros,
+                                        causal=causal, out_dtype=out_dtype)
+        assert fa.fa_check_status() == fa.FA_OK
+        assert (o == 0).all() and torch.isneginf(lse).all()
+
+
 def test_shared_and_expanded_masks(cuda_device):
     """One [Tq, Tk] mask for every (b, h), and a mask expanded over the batch (stride 0)."""
     B, H, L, d = 2, 2, 640, 64
