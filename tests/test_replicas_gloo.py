@@ -63,25 +63,3 @@ def test_single_process_reductions_are_identity():
     assert bench.attn_flops(4, 16, 4096, 4096, 128, True) == 274877906944.0
     assert bench.attn_flops(2, 16, 8192, 8192, 128, True, backward=True) == 2.5 * 549755813888.0
 
-
-def test_blocksparse_pair_count_matches_brute_force():
-    """The benchmark's work count for the block-sparse forward against counting every permitted
-    (query, key) pair one by one, on ragged lengths, causal (Lq < Lk) and not."""
-    import numpy as np
-
-    import bench
-
-    rng = np.random.default_rng(3)
-    for Lq, Lk, causal, blk in ((37, 50, True, 8), (37, 50, False, 8), (64, 64, True, 16), (5, 9, True, 4)):
-        tq, tk = -(-Lq // blk), -(-Lk // blk)
-        mask = (rng.random((2, tq, tk)) < 0.6).astype(np.uint8)
-        want = 0
-        for h in range(2):
-            for i in range(Lq):
-                for j in range(Lk):
-                    if mask[h, i // blk, j // blk] and (not causal or j <= i + Lk - Lq):
-                        want += 1
-        assert bench.blocksparse_pairs(mask, Lq, Lk, causal, blk) == want
-    # the benchmark's shape: a full causal mask at L = 16384 counts L (L + 1) / 2 pairs
-    t = 16384 // 128
-    assert bench.blocksparse_pairs(np.tril(np.ones((t, t))), 16384, 16384, True) == 16384 * 16385 / 2
