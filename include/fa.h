@@ -35,6 +35,14 @@
  *               device, 16-byte aligned.  The caller owns every buffer; the
  *               library never allocates, frees or synchronises.  Calls are
  *               asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   Workspace   A workspace holds one call's scratch from its launch until its
+ *               kernels finish: calls that may run at the same time (on different
+ *               streams) need different workspaces.
+ *   Forwards    fa_forward, fa_forward_varlen and fa_forward_blocksparse claim work
+ *               from one of 256 per-device counters, taken round-robin per call and
+ *               reset by the call's last block; up to 256 forward calls may be in
+ *               flight at once.  A captured CUDA graph keeps its counter, so one
+ *               graph must not be replayed on two streams at the same time.
  *   Devices     Compute capability 10.0 (sm_100a) only; elsewhere calls return
  *               FA_ERR_DEVICE.  There is no fallback path.
  *   Errors      Argument errors are returned synchronously and nothing is
