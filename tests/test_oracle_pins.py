@@ -222,12 +222,14 @@ def test_decode_equals_forward_over_prefix_and_edge_lengths():
 # --- backward --------------------------------------------------------------------------
 
 @pytest.mark.parametrize("causal", [False, True])
-def test_backward_matches_finite_differences(causal):
+@pytest.mark.parametrize("Lq,Lk", [(6, 6), (4, 7)])
+def test_backward_matches_finite_differences(causal, Lq, Lk):
     """Central differences (eps = 1e-6, double) of f = sum(G * O) with respect to
-    every entry of Q, K and V match dQ, dK, dV to 1e-6 relative."""
-    B, H, L, d = 1, 2, 6, 3
-    q, k, v = rnd((B, H, L, d), 27), rnd((B, H, L, d), 28), rnd((B, H, L, d), 29)
-    G = rnd((B, H, L, d), 30)
+    every entry of Q, K and V match dQ, dK, dV to 1e-6 relative; also with fewer
+    queries than keys (bottom-right causal alignment)."""
+    B, H, d = 1, 2, 3
+    q, k, v = rnd((B, H, Lq, d), 27), rnd((B, H, Lk, d), 28), rnd((B, H, Lk, d), 29)
+    G = rnd((B, H, Lq, d), 30)
     scale = 0.8
     dq, dk, dv, _ = oracle.backward(q, k, v, G, scale, causal)
 
