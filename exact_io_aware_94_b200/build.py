@@ -1,6 +1,11 @@
 """Build the C-ABI shared library ``libfa_sm100.so`` in-tree with nvcc (sm_100a only).
 
-Usage: ``python -m exact_io_aware_94_b200.build [--force] [--verbose-ptxas]``.
+Usage: ``python -m exact_io_aware_94_b200.build [--force] [--verbose-ptxas] [--test-hooks]``.
+
+``--test-hooks`` builds ``libfa_sm100_testhooks.so`` instead: the same sources
+compiled with ``FA_TEST_HOOKS``, which shortens every bounded wait to 20 ms and
+exports ``fa_test_inject_fault``, so the tests can make a wait run out.  The
+product library never contains the hooks.
 """
 from __future__ import annotations
 
@@ -17,6 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libfa_sm100.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
+TEST_LIB_PATH = os.path.join(PKG, "libfa_sm100_testhooks.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -37,21 +43,24 @@ def _inputs():
         glob.glob(os.path.join(INCLUDE, "*.h"))
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
+def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = None, test_hooks: bool = False) -> str:
+    out_path = TEST_LIB_PATH if test_hooks else LIB_PATH
+    if not force and up_to_date(out_path):
+        return out_path
     nvcc = nvcc_path()
-    objdir = os.path.join(PKG, "_build")
+    objdir = os.path.join(PKG, "_build_testhooks" if test_hooks else "_build")
     os.makedirs(objdir, exist_ok=True)
     common = ARCH_FLAGS + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I" + INCLUDE, "-I" + CSRC,
                            "--expt-relaxed-constexpr"]
+    if test_hooks:
+        common += ["-DFA_TEST_HOOKS"]
     if verbose_ptxas:
         common += ["-Xptxas", "-v"]
     objs = []
@@ -71,15 +80,16 @@ def build(force: bool = False, verbose_ptxas: bool = False, jobs: int | None = N
             sys.stderr.write("nvcc failed on %s\n" % src)
     if failed:
         raise RuntimeError("CUDA build failed")
-    tmp = LIB_PATH + ".tmp%d" % os.getpid()
+    tmp = out_path + ".tmp%d" % os.getpid()
     subprocess.check_call([nvcc, "-shared", "-o", tmp] + objs + ARCH_FLAGS + ["-Xcompiler", "-fPIC"])
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, out_path)
+    return out_path
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--verbose-ptxas", action="store_true")
+    ap.add_argument("--test-hooks", action="store_true")
     a = ap.parse_args()
-    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas))
+    print(build(force=a.force, verbose_ptxas=a.verbose_ptxas, test_hooks=a.test_hooks))

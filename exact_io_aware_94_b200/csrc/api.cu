@@ -6,8 +6,8 @@
 
 #include <cmath>
 #include <cstdint>
-#include <atomic>
 #include <mutex>
+#include <unordered_map>
 
 #include "fa_internal.h"
 
@@ -15,8 +15,10 @@ namespace fa {
 namespace {
 
 __device__ int g_status;  // one per device; kernels record device-side conditions here
-// Forward unit schedulers: (ticket, finished-CTA count) pairs, used round-robin by
-// launches and reset to zero by the last CTA of each launch.
+// Forward unit schedulers: (ticket, finished-CTA count) pairs.  Each stream gets
+// its own pair the first time it launches a forward (launches on one stream run
+// one after another, so they never share a pair while running), and the last CTA
+// of each launch returns its pair to zero.
 constexpr unsigned kSchedSlots = 256;
 __device__ unsigned int g_fwd_sched[2 * kSchedSlots];
 
@@ -28,7 +30,8 @@ struct DeviceState {
     int num_sms = 0;
     int* status_ptr = nullptr;
     unsigned int* sched_ptr = nullptr;
-    std::atomic<unsigned> sched_next{0};
+    // stream (by its process-unique id) -> scheduler pair; pairs are never handed back
+    std::unordered_map<unsigned long long, unsigned> stream_slot;
 };
 
 std::mutex g_mu;
@@ -71,6 +74,30 @@ int device_state(DeviceState** out) {
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     *out = &st;
+    return FA_OK;
+}
+
+// Scheduler counters for a forward launch on `stream`, or null for the static
+// deal (each CTA takes a fixed, snake-ordered share of the units).  The static
+// deal is used while the stream is being captured into a graph -- a graph may
+// later be replayed on any stream, also on several at once -- and for streams
+// beyond the first kSchedSlots that launched a forward on this device.  Streams
+// are told apart by cudaStreamGetId, which never repeats within a process, so a
+// stream created with the handle of a destroyed one gets a pair of its own.
+int fwd_sched(DeviceState* st, cudaStream_t stream, unsigned int** out) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return FA_ERR_CUDA;
+    *out = nullptr;
+    if (cs != cudaStreamCaptureStatusNone) return FA_OK;
+    unsigned long long id = 0;
+    if (cudaStreamGetId(stream, &id) != cudaSuccess) return FA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = st->stream_slot.find(id);
+    if (it == st->stream_slot.end()) {
+        if (st->stream_slot.size() >= kSchedSlots) return FA_OK;
+        it = st->stream_slot.emplace(id, static_cast<unsigned>(st->stream_slot.size())).first;
+    }
+    *out = st->sched_ptr + 2 * it->second;
     return FA_OK;
 }
 
@@ -149,6 +176,59 @@ int encode_packed_map(CUtensorMap* map, const void* base, int total, int H, int 
     return encode_packed_map_impl(map, base, total, H, d, box_rows, elem_bytes);
 }
 
+// Argument checks of the backward entry points (everything but the scratch).
+int bwd_check_args(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                   const void* dq, const void* dk, const void* dv, int B, int H, int Lq, int Lk, int d, float scale,
+                   int causal, int o_dtype) {
+    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
+    if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
+    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
+    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+        return FA_ERR_INVALID_ARG;
+    const long long bh = static_cast<long long>(B) * H;
+    if (bh * ((Lq + 127) / 128) > 0x7FFFFFFFLL || bh * ((Lk + 127) / 128) > 0x7FFFFFFFLL ||
+        bh * Lq * (d / 8) / 256 > 0x7FFFFFFFLL)
+        return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+// Encodes the maps and launches the backward kernels; dsum is the scratch for D.
+int bwd_launch_checked(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                       void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                       int o_dtype, float* dsum, cudaStream_t stream) {
+    DeviceState* st = nullptr;
+    int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    BwdParams p{};
+    const int BH = B * H;
+    if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, 128)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_do, dO, BH, Lq, d, 128)) != FA_OK) return rc;
+    p.o = o;
+    p.dO = dO;
+    p.lse = lse;
+    p.dsum = dsum;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.status = st->status_ptr;
+    p.B = B;
+    p.H = H;
+    p.Lq = Lq;
+    p.Lk = Lk;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    p.causal = causal ? 1 : 0;
+    p.o_dtype = o_dtype;
+    const cudaError_t e = launch_bwd(p, d, stream);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace fa
 
 using namespace fa;
@@ -201,8 +281,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     p.o = o;
     p.lse = lse;
     p.status = st->status_ptr;
-    // Launches in flight at the same time use different scheduler slots.
-    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    if ((rc = fwd_sched(st, static_cast<cudaStream_t>(stream), &p.sched)) != FA_OK) return rc;
     p.B = B;
     p.H = H;
     p.Lq = Lq;
@@ -272,7 +351,7 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
     p.o = o;
     p.lse = lse;
     p.status = st->status_ptr;
-    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    if ((rc = fwd_sched(st, static_cast<cudaStream_t>(stream), &p.sched)) != FA_OK) return rc;
     p.bs_meta = plan.meta;
     p.bs_list = plan.list;
     p.bs_own = plan.own;
@@ -340,50 +419,12 @@ size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d) {
 int fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
                 void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
                 int o_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
-    if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
-    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dO, 16) ||
-        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
-        return FA_ERR_INVALID_ARG;
-    const long long bh = static_cast<long long>(B) * H;
-    if (bh * ((Lq + 127) / 128) > 0x7FFFFFFFLL || bh * ((Lk + 127) / 128) > 0x7FFFFFFFLL ||
-        bh * Lq * (d / 8) / 256 > 0x7FFFFFFFLL)
-        return FA_ERR_INVALID_ARG;
+    int rc = bwd_check_args(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, o_dtype);
+    if (rc != FA_OK) return rc;
     if (!workspace || !aligned(workspace, 256) || workspace_bytes < bwd_workspace_bytes(B, H, Lq))
         return FA_ERR_WORKSPACE;
-
-    DeviceState* st = nullptr;
-    int rc = device_state(&st);
-    if (rc != FA_OK) return rc;
-
-    BwdParams p{};
-    const int BH = B * H;
-    if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_do, dO, BH, Lq, d, 128)) != FA_OK) return rc;
-    p.o = o;
-    p.dO = dO;
-    p.lse = lse;
-    p.dsum = static_cast<float*>(workspace);
-    p.dq = dq;
-    p.dk = dk;
-    p.dv = dv;
-    p.status = st->status_ptr;
-    p.B = B;
-    p.H = H;
-    p.Lq = Lq;
-    p.Lk = Lk;
-    p.scale = scale;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.causal = causal ? 1 : 0;
-    p.o_dtype = o_dtype;
-    cudaError_t e = launch_bwd(p, d, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    return bwd_launch_checked(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, o_dtype,
+                              static_cast<float*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
 int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,
@@ -417,7 +458,7 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
     p.o = o;
     p.lse = lse;
     p.status = st->status_ptr;
-    p.sched = st->sched_ptr + 2 * (st->sched_next.fetch_add(1, std::memory_order_relaxed) % kSchedSlots);
+    if ((rc = fwd_sched(st, static_cast<cudaStream_t>(stream), &p.sched)) != FA_OK) return rc;
     p.cu_q = cu_seqlens_q;
     p.cu_k = cu_seqlens_k;
     p.max_pairs = static_cast<int>(max_pairs);
@@ -495,12 +536,32 @@ int fa_check_status(void* stream) {
     DeviceState* st = nullptr;
     int rc = device_state(&st);
     if (rc != FA_OK) return rc;
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    (void)stream;  // the status word is per device: wait for every stream of it
+    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
     int h = 0;
     if (cudaMemcpy(&h, st->status_ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
-    if (h != 0 && cudaMemset(st->status_ptr, 0, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
-    if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    if (h != 0) {
+        if (cudaMemset(st->status_ptr, 0, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+    }
     return h;
 }
+
+#ifdef FA_TEST_HOOKS
+// Fault injection for the tests of the bounded waits; exported by the test build
+// (libfa_sm100_testhooks.so) only.  where: 1 = forward K tile, 2 = dK/dV K/V
+// tiles, 3 = paged-decode stage.  Arms a one-shot fault on the current device.
+int fa_test_inject_fault(int where) {
+    DeviceState* st = nullptr;
+    const int rc = device_state(&st);
+    if (rc != FA_OK) return rc;
+    cudaError_t e = cudaErrorInvalidValue;
+    if (where == 1) e = fwd_test_arm_skip_k();
+    else if (where == 2) e = bwd_test_arm_skip_kv();
+    else if (where == 3) e = paged_test_arm_skip_stage();
+    else return FA_ERR_INVALID_ARG;
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"

@@ -30,6 +30,13 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+#ifdef FA_TEST_HOOKS
+// One-shot fault (test build only): the next dK/dV CTA's K and V tiles are not
+// loaded (neither the expected byte count nor the copies), so the MMA warp's
+// wait for them runs out.
+__device__ int g_test_skip_kv;
+#endif
+
 template <int D>
 struct BwdTiles {
     static constexpr int kBoxBytes = 128 * 64 * 2;
@@ -152,14 +159,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
     if (warp == 8) {
         // ================= producer: K, V once; then Q, dO, LSE, D per query tile
         int issued = 0;
+        bool kv_skipped = false;  // test build: the K/V copies were never issued
         if (!*abort_flag) {
             if (lane == 0) {
                 tma_prefetch_desc(&p.tm_q);
                 tma_prefetch_desc(&p.tm_do);
-                mbar_arrive_expect_tx(bar_kv, 2 * T::kTileBytes);
-                for (int b = 0; b < T::kBoxes; ++b) {
-                    tma_load_3d(sK + b * T::kBoxBytes, &p.tm_k, bar_kv, b * 64, j0, bh);
-                    tma_load_3d(sV + b * T::kBoxBytes, &p.tm_v, bar_kv, b * 64, j0, bh);
+#ifdef FA_TEST_HOOKS
+                kv_skipped = atomicExch(&g_test_skip_kv, 0) != 0;
+#endif
+                if (!kv_skipped) {
+                    mbar_arrive_expect_tx(bar_kv, 2 * T::kTileBytes);
+                    for (int b = 0; b < T::kBoxes; ++b) {
+                        tma_load_3d(sK + b * T::kBoxBytes, &p.tm_k, bar_kv, b * 64, j0, bh);
+                        tma_load_3d(sV + b * T::kBoxBytes, &p.tm_v, bar_kv, b * 64, j0, bh);
+                    }
                 }
             }
             for (int t = 0; t < nq; ++t) {
@@ -189,8 +202,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
                 issued = t + 1;
             }
         }
-        if (lane == 0 && *abort_flag) {
-            mbar_wait_drain(bar_kv, 0, p.status);
+        // every copy issued here lands before the CTA exits (each barrier is at the
+        // phase of its last copy)
+        if (lane == 0 && issued > 0) {
+            if (!kv_skipped) mbar_wait_drain(bar_kv, 0, p.status);
             for (int t = max(0, issued - S); t < issued; ++t) mbar_wait_drain(&bar_qd[t % S], (t / S) & 1, p.status);
         }
     } else if (warp == 9) {
@@ -495,12 +510,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq(const __grid_constan
                     tma_load_3d_w(sV + s * T::kTileBytes + b * T::kBoxBytes, &p.tm_v, &bar_v[s], b * 64, j * 128, bh);
                 issued = j + 1;
             }
-            if (*abort_flag) {
-                mbar_wait_drain(bar_qd, 0, p.status);
-                for (int j = max(0, issued - S); j < issued; ++j) {
-                    mbar_wait_drain(&bar_k[j % S], (j / S) & 1, p.status);
-                    mbar_wait_drain(&bar_v[j % S], (j / S) & 1, p.status);
-                }
+            // every copy issued here lands before the CTA exits (each barrier is at
+            // the phase of its last copy)
+            mbar_wait_drain(bar_qd, 0, p.status);
+            for (int j = max(0, issued - S); j < issued; ++j) {
+                mbar_wait_drain(&bar_k[j % S], (j / S) & 1, p.status);
+                mbar_wait_drain(&bar_v[j % S], (j / S) & 1, p.status);
             }
         }
     } else if (warp == 9) {
@@ -688,6 +703,13 @@ cudaError_t launch_bwd_d(const BwdParams& p, cudaStream_t stream) {
 }
 
 }  // namespace
+
+#ifdef FA_TEST_HOOKS
+cudaError_t bwd_test_arm_skip_kv() {
+    const int one = 1;
+    return cudaMemcpyToSymbol(g_test_skip_kv, &one, sizeof(int));
+}
+#endif
 
 size_t bwd_workspace_bytes(int B, int H, int Lq) {
     const size_t n = static_cast<size_t>(B) * H * Lq * sizeof(float);

@@ -38,6 +38,13 @@ namespace {
 
 constexpr int kPlanThreads = 1024;
 
+#ifdef FA_TEST_HOOKS
+// One-shot fault (test build only): the next stage a paged-decode copy warp
+// would fill gets neither its expected byte count nor its copies, so the
+// compute warps' wait for it runs out.
+__device__ int g_test_skip_stage;
+#endif
+
 __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
     uint4 r;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -316,6 +323,7 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
     if (warp == 8) {
         // ---------------- copy warp
         int st = 0;  // stages issued
+        int skipped = -1;  // test build: a stage whose copies were never issued
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
             int b, hkv, hg, chunk;
@@ -330,7 +338,14 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
                     if (!ok) break;
                 }
                 const int n = min(kPgStageKeys, end - k0);
-                if (lane == 0) {
+                bool skip = false;
+#ifdef FA_TEST_HOOKS
+                int armed = 0;
+                if (lane == 0) armed = atomicExch(&g_test_skip_stage, 0);
+                skip = __shfl_sync(0xffffffffu, armed, 0) != 0;
+                if (skip) skipped = st;
+#endif
+                if (lane == 0 && !skip) {
                     mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(n) * D * 2 * 2);
                     for (int key = k0; key < k0 + n;) {
                         int pg = table[key >> p.page_shift];
@@ -350,10 +365,10 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
                 __syncwarp();
             }
         }
-        if (*abort_flag) {
-            // copies already issued land before the CTA's shared memory goes away
-            for (int t = max(0, st - kPgStages); t < st; ++t) mbar_wait_drain(&full[t % kPgStages], (t / kPgStages) & 1, p.status);
-        }
+        // every copy issued here lands before the CTA's shared memory goes away
+        // (each barrier is at the phase of its last copy)
+        for (int t = max(0, st - kPgStages); t < st; ++t)
+            if (t != skipped) mbar_wait_drain(&full[t % kPgStages], (t / kPgStages) & 1, p.status);
     } else {
         // ---------------- compute warps 0-7
         const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;
@@ -552,6 +567,13 @@ cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaS
     if (e != cudaSuccess) return e;
     return d == 128 ? launch_paged_d<128>(p, num_sms, stream) : launch_paged_d<64>(p, num_sms, stream);
 }
+
+#ifdef FA_TEST_HOOKS
+cudaError_t paged_test_arm_skip_stage() {
+    const int one = 1;
+    return cudaMemcpyToSymbol(g_test_skip_stage, &one, sizeof(int));
+}
+#endif
 
 size_t decode_workspace_bytes(int B, int H, int cap, int d) {
     const size_t max_splits = (static_cast<size_t>(cap) + kDecodeSplit - 1) / kDecodeSplit;

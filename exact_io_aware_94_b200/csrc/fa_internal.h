@@ -11,8 +11,21 @@
 namespace fa {
 
 // Every bounded wait in a kernel gives up after this long (nanoseconds of
-// %globaltimer), records FA_ERR_TIMEOUT and lets the CTA exit.
+// %globaltimer), records FA_ERR_TIMEOUT and lets the CTA exit.  The fault-
+// injection build used by the tests (FA_TEST_HOOKS) waits 20 ms instead.
+#ifdef FA_TEST_HOOKS
+constexpr uint64_t kWaitTimeoutNs = 20000000ull;
+#else
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
+#endif
+
+#ifdef FA_TEST_HOOKS
+// Fault injection (test build only): arm a one-shot fault in one kernel's
+// producer.  Each returns a CUDA error code.
+cudaError_t fwd_test_arm_skip_k();      // forward: the next K tile a producer would load is never loaded
+cudaError_t bwd_test_arm_skip_kv();     // dK/dV kernel: the next CTA's K/V tiles are never loaded
+cudaError_t paged_test_arm_skip_stage();  // paged decode: the next stage's copies are never issued
+#endif
 
 // Forward kernel tiling: two 128-row Q tiles per CTA (one per softmax
 // warpgroup), 128-key K/V tiles.
@@ -36,7 +49,8 @@ struct __align__(64) FwdParams {
     void* o;
     float* lse;
     int* status;
-    unsigned int* sched;  // [0]: next unit ticket, [1]: CTAs finished; both zero between launches
+    unsigned int* sched;  // [0]: next unit ticket, [1]: CTAs finished; both zero between launches.
+                          // Null: static deal (no counters).
     // packed variable-length batch (fa_forward_varlen): sequence b owns rows [cu_q[b], cu_q[b+1])
     // of q, o [total_q, H, d] and [cu_k[b], cu_k[b+1]) of k, v [total_k, H, d]; Lq = total_q,
     // Lk = total_k, and max_pairs = ceil(max_seqlen_q / 256).  Null for a batched call.
@@ -86,6 +100,12 @@ size_t bwd_workspace_bytes(int B, int H, int Lq);
 
 // Helpers implemented in api.cu for the other entry points.
 int prepare_device(int** status_ptr);
+int bwd_check_args(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                   const void* dq, const void* dk, const void* dv, int B, int H, int Lq, int Lk, int d, float scale,
+                   int causal, int o_dtype);
+int bwd_launch_checked(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                       void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk, int d, float scale, int causal,
+                       int o_dtype, float* dsum, cudaStream_t stream);
 int encode_tile_map(CUtensorMap* map, const void* base, int BH, int L, int d, int box_rows);
 bool shape_ok(int B, int H, int L, int d);
 // Every kernel takes the running maximum over raw scores q.k and applies the

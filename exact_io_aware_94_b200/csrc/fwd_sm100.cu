@@ -8,8 +8,9 @@
 //
 // B200 mapping.  A work unit is 256 query rows of one (b, h): two 128-row Q
 // tiles, one per softmax warpgroup.  The kernel is persistent (one CTA per SM)
-// and claims units one at a time from the launch's ticket counter, in a fixed
-// heavy-first order, so the CTAs finish within a unit of one another.  The
+// and claims units one at a time from its stream's ticket counter, in a fixed
+// heavy-first order, so the CTAs finish within a unit of one another (under
+// graph capture, a static snake-ordered deal of the same order instead).  The
 // producer warp claims each unit and hands it to the other roles through a
 // small ring in shared memory.  Each warpgroup's Q tile of
 // the next unit is loaded as soon as that warpgroup's last S MMA of the current
@@ -51,6 +52,13 @@ namespace {
 
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kUnitRing = 4;  // units published ahead by the producer
+
+#ifdef FA_TEST_HOOKS
+// One-shot fault (test build only): the next K tile a producer would load is
+// skipped -- neither its expected byte count nor its copy is issued -- so the
+// MMA warp's wait for it runs out.
+__device__ int g_test_skip_k;
+#endif
 
 
 
@@ -282,6 +290,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             int kc = 0;                // K/V tiles started so far (ring position)
             int nk = 0, nv = 0;        // K and V tiles whose loads were issued
             int q_iter[2] = {0, 0};    // Q tiles requested per warpgroup
+            unsigned claims = 0;       // units claimed by this CTA (static deal)
+            int skipped_k = -1;        // test build: ring position of a K tile never loaded
             bool ok = true;
             for (int it = 0; ok; ++it) {
                 // claim the next unit (heavy-first order) and publish it
@@ -291,8 +301,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 Unit un;
                 for (;;) {  // a packed batch's virtual units past a sequence's end are skipped here
                     unsigned int ticket = 0;
-                    if (lane == 0) ticket = atomicAdd(p.sched, 1u);
-                    u = static_cast<int>(min(__shfl_sync(0xffffffffu, ticket, 0), static_cast<unsigned>(n_units)));
+                    if (p.sched) {
+                        if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+                        ticket = __shfl_sync(0xffffffffu, ticket, 0);
+                    } else {
+                        // static deal: claim k of CTA c is unit k*G + c, snake-ordered
+                        const unsigned G = gridDim.x, k = claims++;
+                        ticket = k * G + ((k & 1u) ? G - 1u - blockIdx.x : blockIdx.x);
+                    }
+                    u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
                     if (u >= n_units) break;
                     un = get_unit<VARLEN, BSPARSE>(p, u, true);
                     if (!VARLEN || un.n_kv0 > 0 || un.n_kv1 > 0) break;
@@ -329,10 +346,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
                     const int ky = VARLEN ? un.bh % p.H : kvt * kFwdBN;
                     const int kz = VARLEN ? un.k0 + j * kFwdBN : un.bh;
-                    mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
-                    for (int b = 0; b < Lay::kBoxes; ++b)
-                        tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64, ky,
-                                      kz);
+                    bool skip = false;
+#ifdef FA_TEST_HOOKS
+                    int armed = 0;
+                    if (lane == 0) armed = atomicExch(&g_test_skip_k, 0);
+                    skip = __shfl_sync(0xffffffffu, armed, 0) != 0;
+                    if (skip) skipped_k = kc;
+#endif
+                    if (!skip) {
+                        mbar_arrive_expect_tx_w(&bar_k[s], Lay::kTileBytes);
+                        for (int b = 0; b < Lay::kBoxes; ++b)
+                            tma_load_3d_w(sK + s * Lay::kTileBytes + b * Lay::kBoxBytes, &p.tm_k, &bar_k[s], b * 64,
+                                          ky, kz);
+                    }
                     ++nk;
                     if (j == 0 && un.n_kv1 > 0 && !(ok = load_q(1))) break;
                     if (kc >= S && !(ok = wait(&bar_vfree[s], ((kc / S) - 1) & 1))) break;
@@ -343,13 +369,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     ++nv;
                 }
             }
-            if (*abort_flag) {
-                // Let copies already in flight land before the CTA's smem goes away.
-                for (int w = 0; w < 2; ++w)
-                    if (q_iter[w] > 0) mbar_wait_drain(&bar_q[w], (q_iter[w] - 1) & 1, p.status);
-                for (int t = max(0, nk - S); t < nk; ++t) mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
-                for (int t = max(0, nv - S); t < nv; ++t) mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
-            }
+            // Every copy this warp issued lands before the CTA's shared memory goes
+            // away, also when a wait elsewhere in the CTA ran out after this loop
+            // ended.  (Each barrier waited on here is at the phase of its last copy.)
+            for (int w = 0; w < 2; ++w)
+                if (q_iter[w] > 0) mbar_wait_drain(&bar_q[w], (q_iter[w] - 1) & 1, p.status);
+            for (int t = max(0, nk - S); t < nk; ++t)
+                if (t != skipped_k) mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
+            for (int t = max(0, nv - S); t < nv; ++t) mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
         }
     } else if (warp == 9) {
         // ================= MMA issuer =================
@@ -786,7 +813,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     }
     // Every producer of this launch has stopped claiming units once it reaches here;
     // the last CTA to finish returns the scheduler slot to zero for a later launch.
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && p.sched) {
         __threadfence();
         if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
             atomicExch(p.sched, 0u);
@@ -931,6 +958,13 @@ cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p,
     return d == 128 ? launch_fwd_kernel<128, false, true>(p, num_sms, stream)
                     : launch_fwd_kernel<64, false, true>(p, num_sms, stream);
 }
+
+#ifdef FA_TEST_HOOKS
+cudaError_t fwd_test_arm_skip_k() {
+    const int one = 1;
+    return cudaMemcpyToSymbol(g_test_skip_k, &one, sizeof(int));
+}
+#endif
 
 size_t bs_workspace_bytes(int B, int H, int Lq, int Lk) {
     const size_t n_units = static_cast<size_t>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);

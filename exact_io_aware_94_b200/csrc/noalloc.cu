@@ -38,8 +38,6 @@ int scratch_for_current_device(float** out) {
     return FA_OK;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace fa
 
@@ -48,45 +46,15 @@ using namespace fa;
 extern "C" int fa_backward_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
                                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Lq, int Lk,
                                    int d, float scale, int causal, int o_dtype, void* stream) {
-    if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-    if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
-    if (!shape_ok(B, H, Lq, d) || !shape_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
-    if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
-    if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(dq) ||
-        !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u) != 0)
-        return FA_ERR_INVALID_ARG;
-    if (static_cast<long long>(B) * H * Lq > FA_NOALLOC_MAX_ROWS) return FA_ERR_TOO_LARGE;
-
-    int* status = nullptr;
-    int rc = prepare_device(&status);
+    // the same checks as fa_backward, then the one limit of the fixed scratch
+    int rc = bwd_check_args(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, o_dtype);
     if (rc != FA_OK) return rc;
+    if (static_cast<long long>(B) * H * Lq > FA_NOALLOC_MAX_ROWS) return FA_ERR_TOO_LARGE;
+    int* status = nullptr;
+    if ((rc = prepare_device(&status)) != FA_OK) return rc;
     float* scratch = nullptr;
     if ((rc = scratch_for_current_device(&scratch)) != FA_OK) return rc;
-
-    BwdParams p{};
-    const int BH = B * H;
-    if ((rc = encode_tile_map(&p.tm_q, q, BH, Lq, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_tile_map(&p.tm_k, k, BH, Lk, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_tile_map(&p.tm_v, v, BH, Lk, d, 128)) != FA_OK) return rc;
-    if ((rc = encode_tile_map(&p.tm_do, dO, BH, Lq, d, 128)) != FA_OK) return rc;
-    p.o = o;
-    p.dO = dO;
-    p.lse = lse;
-    p.dsum = scratch;  // the pre-kernel writes every D_i before the main kernels read it
-    p.dq = dq;
-    p.dk = dk;
-    p.dv = dv;
-    p.status = status;
-    p.B = B;
-    p.H = H;
-    p.Lq = Lq;
-    p.Lk = Lk;
-    p.scale = scale;
-    p.scale_log2 = scale * 1.4426950408889634f;
-    p.causal = causal ? 1 : 0;
-    p.o_dtype = o_dtype;
-    const cudaError_t e = launch_bwd(p, d, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    // the pre-kernel writes every D_i before the main kernels read it
+    return bwd_launch_checked(q, k, v, o, dO, lse, dq, dk, dv, B, H, Lq, Lk, d, scale, causal, o_dtype, scratch,
+                              static_cast<cudaStream_t>(stream));
 }

@@ -321,31 +321,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t packed) { return __uint_as_float(packed << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t packed) { return __uint_as_float(packed & 0xFFFF0000u); }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-    float d;
-    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-    return d;
-}
-
-// 2^x on the FMA pipe instead of MUFU.  Cody-Waite style range reduction:
-// n = round(x) by the 1.5*2^23 magic-number addition (n lands in the low
-// mantissa bits), f = x - n in [-1/2, 1/2], 2^f by a degree-3 polynomial fitted
-// here to minimise relative error on [-1/2, 1/2] (max about 7.5e-5, far below
-// the bf16 rounding P~ gets next), then n is added to the exponent field.
-// x is clamped to [-126, +inf) so the exponent cannot wrap; callers keep x <= 9.
-__device__ __forceinline__ float exp2_poly(float x) {
-    const float xc = fmaxf(x, -126.0f);
-    const float j = xc + 12582912.0f;           // bits: 0x4B400000 + round(x)
-    const float f = xc - (j - 12582912.0f);     // x - round(x)
-    float p = fmaf(0.055170975625514984f, f, 0.24260970950126648f);
-    p = fmaf(p, f, 0.6932609677314758f);
-    p = fmaf(p, f, 0.9999281764030457f);
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(j) << 23));
-}
-
 // Value of x after rounding to bf16 (nearest-even), as a float.
 __device__ __forceinline__ float round_bf16(float x) { return __uint_as_float(pack_bf16x2(x, 0.0f) << 16); }
-
-__device__ __forceinline__ int elect_one_lane() { return (threadIdx.x & 31) == 0; }
 
 }  // namespace fa

@@ -38,13 +38,20 @@
  *   Workspace   A workspace holds one call's scratch from its launch until its
  *               kernels finish: calls that may run at the same time (on different
  *               streams) need different workspaces.
- *   Forwards    fa_forward, fa_forward_varlen and fa_forward_blocksparse claim work
- *               from one of 256 per-device counters, taken round-robin per call and
- *               reset by the call's last block; up to 256 forward calls may be in
- *               flight at once.  A captured CUDA graph keeps its counter, so one
- *               graph must not be replayed on two streams at the same time.
+ *   Forwards    fa_forward, fa_forward_varlen and fa_forward_blocksparse hand out
+ *               their work units from a per-stream counter (each of the first 256
+ *               streams that launch a forward on a device gets its own; calls on
+ *               one stream run one after another, and each call's last block
+ *               returns the counter to zero).  While `stream` is being captured
+ *               into a CUDA graph, and on streams beyond the first 256, a call
+ *               deals its units statically instead, so a captured graph may be
+ *               replayed on any number of streams at once.
  *   Devices     Compute capability 10.0 (sm_100a) only; elsewhere calls return
- *               FA_ERR_DEVICE.  There is no fallback path.
+ *               FA_ERR_DEVICE.  There is no fallback path.  The library looks up
+ *               the device addresses of its static arrays (status word, forward
+ *               counters, fa_backward_noalloc's scratch) once per device and keeps
+ *               them, so resetting a device (cudaDeviceReset) while the library is
+ *               loaded is not supported.
  *   Errors      Argument errors are returned synchronously and nothing is
  *               launched.  A failed launch returns FA_ERR_CUDA.  Conditions met
  *               on the device (a bounded wait that ran out, a cache length outside
@@ -250,9 +257,16 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
                            size_t workspace_bytes, void* stream);
 
 /*
- * Synchronises `stream`, returns the current device's status word (FA_OK if no
- * kernel recorded a condition since the last call) and clears it.  Returns
- * FA_ERR_CUDA if the synchronisation itself fails.
+ * Synchronises the whole current device (every stream: the status word is shared
+ * by all of them), then returns the device's status word (FA_OK if no kernel
+ * recorded a condition since the last call) and clears it.  `stream` is not used.
+ * Returns FA_ERR_CUDA if the synchronisation itself fails.  Must not be called
+ * while a stream of the device is being captured.
+ *
+ * After FA_ERR_TIMEOUT has been recorded, every later kernel of this library on
+ * the device sees it when it starts and exits at once without writing its
+ * outputs (the calls still return FA_OK); calls compute again once
+ * fa_check_status() has returned and cleared the condition.
  */
 int fa_check_status(void* stream);
 
