@@ -217,6 +217,45 @@ def oracle_forward_sample(workload, budget_s, seed=0):
     return f / t / 1e12, t, oracle.num_threads(), desc
 
 
+def oracle_tiny_full():
+    """Time the oracle on the whole tiny forward (B=1 H=2 L=256 d=64, non-causal):
+    returns (tflops, seconds)."""
+    import oracle
+    from exact_io_aware_94_b200.inputs import WORKLOADS, attention_inputs
+
+    w = WORKLOADS["tiny_fwd"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    inp = attention_inputs(B, H, L, L, d, seed=w["seed"])
+    flops = attn_flops(B, H, L, L, d, w["causal"])
+    reps, t = 0, 0.0
+    t0 = time.perf_counter()
+    while t < 0.5:
+        oracle.forward(inp.q, inp.k, inp.v, 1.0 / math.sqrt(d), w["causal"])
+        reps += 1
+        t = time.perf_counter() - t0
+    return flops * reps / t / 1e12, t / reps
+
+
+def cpu_baseline(budget_s):
+    """The oracle on the host cores (all of them, then one): the headline workload's
+    row sample, and the whole tiny forward."""
+    import oracle
+
+    tf, _, cores, desc = oracle_forward_sample(HEADLINE, budget_s)
+    out = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+    tiny_tf, tiny_s = oracle_tiny_full()
+    out["tiny_fwd_full"] = {"TFLOP/s": tiny_tf, "s_per_call": tiny_s, "cores": cores}
+    oracle.set_num_threads(1)
+    try:
+        tf1, _, _, desc1 = oracle_forward_sample(HEADLINE, budget_s / 4)
+        tiny_tf1, tiny_s1 = oracle_tiny_full()
+    finally:
+        oracle.set_num_threads(cores)
+    out["single_core"] = {"cores": 1, HEADLINE: {"TFLOP/s": tf1, "sample": desc1},
+                          "tiny_fwd_full": {"TFLOP/s": tiny_tf1, "s_per_call": tiny_s1}}
+    return out
+
+
 # ----------------------------------------------------------------------------- GPU timing
 def time_steps(fn, steps, warmup, stream, dist=None, device=None):
     """Warm up, then time exactly `steps` calls between barrier+synchronize pairs with
@@ -362,8 +401,7 @@ def run_ours(args, dist, rank, world, device):
         "legs": legs,
     }
     if rank == 0 and world == 1 and args.cpu_baseline:
-        tf, secs_cpu, cores, desc = oracle_forward_sample(HEADLINE, args.cpu_budget)
-        out["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        out["cpu_baseline"] = cpu_baseline(args.cpu_budget)
     return out
 
 
@@ -373,6 +411,25 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
     legs = {}
     steps = max(3, min(args.steps, 20))
     warm = max(3, args.warmup)
+
+    # the tiny forward (B=1 H=2 L=256 d=64, non-causal): latency-bound, so no roofline
+    w = WORKLOADS["tiny_fwd"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    gen = torch.Generator(device=device).manual_seed(w["seed"] + 1000 * rank)
+    q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=device)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=device)
+
+    def fwd_tiny():
+        rc = fa.fa_forward(q, k, v, o, lse, B, H, L, L, d, 1.0 / math.sqrt(d), 0, fa.FA_DT_F32, stream)
+        assert rc == fa.FA_OK
+
+    t_t = time_steps(fwd_tiny, steps, warm, stream, dist, device) / steps
+    legs["tiny_fwd"] = {"ms": round(t_t * 1e3, 5), "us": round(t_t * 1e6, 2),
+                        "TFLOP/s": round(attn_flops(B, H, L, L, d, False) / t_t / 1e12, 3), "launches": 1,
+                        "note": "latency-bound (4 units on 148 SMs): time reported, no roofline target",
+                        "l2": "inputs 192 KB, L2-resident between calls"}
+    del q, k, v, o, lse
 
     # training forward + backward at L = 8192
     w = WORKLOADS["train_L8192"]

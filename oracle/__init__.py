@@ -72,6 +72,8 @@ def _load():
         lib.oracle_merge.argtypes = [dp, dp, i64, i64, dp, dp]
         lib.oracle_num_threads.restype = c_int
         lib.oracle_num_threads.argtypes = []
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [c_int]
         _lib = lib
     return _lib
 
@@ -285,3 +287,8 @@ def merge(o_parts, lse_parts):
 def num_threads() -> int:
     """OpenMP threads the oracle's parallel regions use."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads for the oracle's later parallel regions (timing only: results do not depend on it)."""
+    _load().oracle_set_num_threads(int(n))

@@ -550,3 +550,12 @@ int oracle_num_threads(void) {
     }
     return n;
 }
+
+/* Threads of the following parallel regions (timing only; results do not depend on it). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -7,7 +7,7 @@ import torch
 
 import exact_io_aware_94_b200 as fa
 import oracle
-from exact_io_aware_94_b200.inputs import varlen_inputs
+from exact_io_aware_94_b200.inputs import WORKLOADS, varlen_inputs
 
 from .parity import check_lse, check_o, check_o_bf16
 
@@ -90,3 +90,48 @@ def test_varlen_invalid_sequence_is_skipped_and_flagged(cuda_device):
     o_ref, lse_ref = oracle.forward_varlen(q_k, k_k, v_k, cu, cu, 1.0 / math.sqrt(d), True)
     check_o(o[keep], o_ref, "varlen O (kept sequences)")
     check_lse(lse[:, keep], lse_ref, "varlen LSE (kept sequences)")
+
+
+@pytest.mark.slow
+def test_varlen_benchmark_workload_sampled_rows(cuda_device):
+    """The packed prefill batch the benchmark times (16 causal sequences with
+    lengths U[512, 8192] from the workload's seed, H16, d128; up to 32 pairs of
+    query tiles and 64 key tiles per unit), with O prefilled with NaN: every row
+    must be written, and sampled rows of every (sequence, head) must match the
+    oracle.  The sample holds each sequence's first and last rows, the rows on
+    both sides of the 128- and 256-row tile boundaries of several units, every
+    row of the last partial 32-row box (written row by row), and random rows."""
+    w = WORKLOADS["prefill_varlen"]
+    B, H, d = w["B"], w["H"], w["d"]
+    cg = torch.Generator("cpu").manual_seed(w["seed"])
+    lens = [int(x) for x in torch.randint(w["len_lo"], w["len_hi"] + 1, (B,), generator=cg)]
+    inp = varlen_inputs(lens, lens, H, d, seed=w["seed"])
+    o, lse = run(inp, H, d, True, torch.float32, cuda_device)
+    assert fa.fa_check_status() == fa.FA_OK
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    scale = 1.0 / math.sqrt(d)
+    rng = np.random.default_rng(w["seed"])
+    cu = inp.cu_q.tolist()
+    n_checked = 0
+    for b, L in enumerate(lens):
+        fixed = {0, 1, L - 1}
+        for u in (0, 1, L // 512, (L - 1) // 256):
+            for r in (u * 256 - 1, u * 256, u * 256 + 127, u * 256 + 128):
+                fixed.add(r)
+        fixed.update(range(L - L % 32, L))  # the last partial 32-row box (empty when L % 32 == 0)
+        fixed = sorted(r for r in fixed if 0 <= r < L)
+        # one sequence as a batched [1, H, L, d] problem for the oracle
+        qb, kb, vb = (t[cu[b]:cu[b + 1]].permute(1, 0, 2).unsqueeze(0).contiguous() for t in (inp.q, inp.k, inp.v))
+        rows = []
+        for h in range(H):
+            pick = set(fixed) | set(rng.integers(0, L, size=16).tolist())
+            rows += [h * L + r for r in sorted(pick)]
+        rows = np.array(rows, dtype=np.int64)
+        o_ref, lse_ref = oracle.forward_rows(qb, kb, vb, rows, scale, True)
+        h_idx, r_idx = rows // L, rows % L
+        tok = torch.as_tensor(cu[b] + r_idx, device=cuda_device)
+        hh = torch.as_tensor(h_idx, device=cuda_device)
+        check_o(o[tok, hh], o_ref, "varlen benchmark workload O (sequence %d)" % b)
+        check_lse(lse[hh, tok], lse_ref, "varlen benchmark workload LSE (sequence %d)" % b)
+        n_checked += rows.size
+    assert n_checked >= 256 * H
