@@ -19,13 +19,18 @@
 // consecutive units overlap.
 //   warp 8      TMA producer: Q tiles per unit, K_j / V_j through a smem ring.
 //   warp 9      MMA issuer: S_w = Q_w K_j^T into TMEM (SS MMA),
-//               O_w += P_w V_j with P_w read from TMEM (TS MMA).
-//               In both warps the whole warp runs the control flow and one
-//               lane chosen by elect.sync issues each copy or MMA: the
-//               operands then stay warp-uniform, which keeps the issue cost
-//               per MMA well under the MMA's own 64 cycles.
-//   warps 10-11 idle (they complete the third warpgroup, whose registers
-//               setmaxnreg hands to the softmax warpgroups).
+//               O_w += P_w V_j with P_w read from TMEM (TS MMA), for both
+//               warpgroups in a fixed alternating order.
+//   warps 9, 10 block-sparse kernel only: one MMA issuer per softmax
+//               warpgroup (w = warp - 9), so a query block whose key-block
+//               list is shorter or sparser never waits behind the other's
+//               entries; the two meet only at the K/V ring.
+//               In the producer and issuer warps the whole warp runs the
+//               control flow and one lane chosen by elect.sync issues each
+//               copy or MMA: the operands then stay warp-uniform, which keeps
+//               the issue cost per MMA well under the MMA's own 64 cycles.
+//   warps 10-11 otherwise idle (they complete the third warpgroup, whose
+//               registers setmaxnreg hands to the softmax warpgroups).
 //   warps 0-3   softmax warpgroup 0 (rows 0..127 of the unit), warps 4-7
 //               warpgroup 1 (rows 128..255).  One thread owns one row: it loads
 //               its score row from TMEM, applies the mask, updates m and l,
@@ -72,13 +77,14 @@ struct FwdLayout {
     static constexpr int kKOff = kQOff + 2 * kTileBytes;
     static constexpr int kVOff = kKOff + kStages * kTileBytes;
     static constexpr int kBarOff = kVOff + kStages * kTileBytes;
-    // barriers: q[2], q_free[2], k[S], v[S], k_free[S], v_free[S], s[2], p[2][2 halves], o[2], o_free[2], drain
-    static constexpr int kNumBars = 4 + 4 * kStages + 10 + 1 + 2 * 4;  // + unit ring full/free
+    // barriers: q[2], q_free[2], k[S], v[S], k_free[S], v_free[S], s[2], p[2][2 halves], o[2], o_free[2],
+    // drain[2]
+    static constexpr int kNumBars = 4 + 4 * kStages + 10 + 2 + 2 * 4;  // + unit ring full/free
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // epilogue staging for the O tile stores: 4 KB per softmax warp (32 rows x 128 bytes,
     // 128-byte swizzle, so 1024-byte aligned)
-    static constexpr int kRingOff = kMiscOff + 16;  // 4 unit indices
-    static constexpr int kStageOff = (kRingOff + 16 + 1023) / 1024 * 1024;
+    static constexpr int kRingOff = kMiscOff + 16;  // 4 unit indices, then (block-sparse) 4 int4 unit metadata
+    static constexpr int kStageOff = (kRingOff + 16 + 64 + 1023) / 1024 * 1024;
     static constexpr int kBytes = kStageOff + 8 * 4096 + 1024;  // + alignment slack
 };
 
@@ -170,14 +176,15 @@ __device__ __forceinline__ size_t bsparse_index(const FwdParams& p, int bh, int 
     return static_cast<size_t>(bh) * n_pairs + i0 / kFwdRowsPerCta;
 }
 
-__device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u) {
+// meta: the unit's bs_meta entry (its first field is the union-list length).
+__device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u, const int4& meta) {
     const int BH = p.B * p.H;
     const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
     Unit r;
     const int pair = n_pairs - 1 - u / BH;
     r.bh = u % BH;
     r.i0 = pair * kFwdRowsPerCta;
-    const int cnt = p.bs_meta[bsparse_index(p, r.bh, r.i0)].x;
+    const int cnt = meta.x;
     r.n_kv0 = cnt;
     r.n_kv1 = (r.i0 + kFwdBM < p.Lq) ? cnt : 0;
     r.q0 = 0;
@@ -192,12 +199,38 @@ __device__ __forceinline__ const uint16_t* bsparse_list(const FwdParams& p, cons
     return p.bs_list + bsparse_index(p, un.bh, un.i0) * p.bs_tk;
 }
 
+// Unit u; block-sparse units need their metadata (meta), which the producer
+// reads once and publishes with the unit.
 template <bool VARLEN, bool BSPARSE>
-__device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag) {
+__device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag, const int4& meta) {
     if constexpr (VARLEN) return unit_of_varlen(p, u, flag);
-    else if constexpr (BSPARSE) return unit_of_bsparse(p, u);
+    else if constexpr (BSPARSE) return unit_of_bsparse(p, u, meta);
     else return unit_of(p, u);
 }
+
+// The block-sparse metadata of unit u (read by the producer only).
+__device__ __forceinline__ int4 bsparse_meta_of(const FwdParams& p, int u) {
+    const int BH = p.B * p.H;
+    const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
+    return __ldg(p.bs_meta + bsparse_index(p, u % BH, (n_pairs - 1 - u / BH) * kFwdRowsPerCta));
+}
+
+// Entry j of a unit's key-block list, read 32 entries at a time by the whole
+// warp (one coalesced load per 32 entries) and handed out by shuffle.  j must be
+// warp-uniform and visited in increasing order; n is the list's length.
+struct ListWindow {
+    int base = -32;
+    uint32_t ent = 0;
+    __device__ __forceinline__ int get(const uint16_t* lst, int j, int n) {
+        const int b = j & ~31;
+        if (b != base) {
+            base = b;
+            const int lane = threadIdx.x & 31;
+            ent = (b + lane < n) ? __ldg(lst + b + lane) : 0u;
+        }
+        return static_cast<int>(__shfl_sync(0xffffffffu, ent, j & 31));
+    }
+};
 
 template <int D, bool VARLEN, bool BSPARSE>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_constant__ FwdParams p) {
@@ -221,12 +254,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint64_t* bar_p = bar_s + 2;  // [2 * w + half]
     uint64_t* bar_o = bar_p + 4;
     uint64_t* bar_ofree = bar_o + 2;
-    uint64_t* bar_drain = bar_ofree + 2;
+    uint64_t* bar_drain = bar_ofree + 2;  // [i]: MMA issuer i's last MMAs are done
     // Unit ring: the producer claims units from the launch's ticket counter and
-    // publishes them here; the MMA warp and the 8 softmax warps read each entry.
-    uint64_t* bar_ufull = bar_drain + 1;
+    // publishes them here; the MMA warp(s) and the 8 softmax warps read each entry.
+    uint64_t* bar_ufull = bar_drain + 2;
     uint64_t* bar_ufree = bar_ufull + kUnitRing;
     volatile int* s_unit = reinterpret_cast<volatile int*>(smem + Lay::kRingOff);
+    int4* s_meta = reinterpret_cast<int4*>(smem + Lay::kRingOff + 16);  // block-sparse unit metadata
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -243,8 +277,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
         for (int s = 0; s < S; ++s) {
             mbar_init(&bar_k[s], 1);
             mbar_init(&bar_v[s], 1);
-            mbar_init(&bar_kfree[s], 1);
-            mbar_init(&bar_vfree[s], 1);
+            // block-sparse: one arrival from each of the two MMA issuers
+            mbar_init(&bar_kfree[s], BSPARSE ? 2 : 1);
+            mbar_init(&bar_vfree[s], BSPARSE ? 2 : 1);
         }
         for (int w = 0; w < 2; ++w) {
             mbar_init(&bar_s[w], 1);
@@ -253,10 +288,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             mbar_init(&bar_o[w], 1);
             mbar_init(&bar_ofree[w], 4 * 32);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(&bar_drain[0], 1);
+        mbar_init(&bar_drain[1], 1);
         for (int r = 0; r < kUnitRing; ++r) {
             mbar_init(&bar_ufull[r], 1);
-            mbar_init(&bar_ufree[r], 1 + 8);  // MMA warp + 8 softmax warps
+            mbar_init(&bar_ufree[r], (BSPARSE ? 2 : 1) + 8);  // MMA warp(s) + 8 softmax warps
         }
         *abort_flag = (atomicAdd(p.status, 0) == FA_ERR_TIMEOUT) ? 1 : 0;
         fence_barrier_init();
@@ -299,6 +335,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 if (it >= kUnitRing && !(ok = wait(&bar_ufree[rs], ((it / kUnitRing) - 1) & 1))) break;
                 int u;
                 Unit un;
+                int4 meta = make_int4(0, 0, 0, 0);
                 for (;;) {  // a packed batch's virtual units past a sequence's end are skipped here
                     unsigned int ticket = 0;
                     if (p.sched) {
@@ -311,11 +348,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     }
                     u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
                     if (u >= n_units) break;
-                    un = get_unit<VARLEN, BSPARSE>(p, u, true);
+                    if constexpr (BSPARSE) meta = bsparse_meta_of(p, u);
+                    un = get_unit<VARLEN, BSPARSE>(p, u, true, meta);
                     if (!VARLEN || un.n_kv0 > 0 || un.n_kv1 > 0) break;
                 }
                 if (lane == 0) {
                     s_unit[rs] = u;
+                    if constexpr (BSPARSE) s_meta[rs] = meta;
                     mbar_arrive(&bar_ufull[rs]);
                 }
                 __syncwarp();
@@ -339,10 +378,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 if (!(ok = load_q(0))) break;
                 const uint16_t* bs_list = nullptr;
                 if constexpr (BSPARSE) bs_list = bsparse_list(p, un);
+                ListWindow lw;
                 for (int j = 0; j < n_max; ++j, ++kc) {
                     const int s = kc % S;
                     int kvt = j;  // key block loaded as the unit's j-th tile
-                    if constexpr (BSPARSE) kvt = __ldg(bs_list + j) & kBsEntryTile;
+                    if constexpr (BSPARSE) kvt = lw.get(bs_list, j, n_max) & kBsEntryTile;
                     if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
                     const int ky = VARLEN ? un.bh % p.H : kvt * kFwdBN;
                     const int kz = VARLEN ? un.k0 + j * kFwdBN : un.bh;
@@ -378,8 +418,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 if (t != skipped_k) mbar_wait_drain(&bar_k[t % S], (t / S) & 1, p.status);
             for (int t = max(0, nv - S); t < nv; ++t) mbar_wait_drain(&bar_v[t % S], (t / S) & 1, p.status);
         }
-    } else if (warp == 9) {
-        // ================= MMA issuer =================
+    } else if (!BSPARSE && warp == 9) {
+        // ================= MMA issuer (dense and packed kernels) =================
+        // One issuer for both warpgroups, in the fixed order PV0(j), S0(j+1), PV1(j),
+        // S1(j+1): the two softmax warpgroups stay half a tile period apart, so their
+        // exponential phases do not collide and the tensor pipe alternates between
+        // them.  (Two free-running issuers measured 9-26% slower here.)
         // The whole warp runs the loop, so descriptors and TMEM addresses are
         // warp-uniform; one elected lane issues each MMA and commit.
         auto wait = [&](uint64_t* bar, uint32_t parity) {
@@ -425,85 +469,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
-                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
-                if constexpr (BSPARSE) {
-                    // Walk the union list; query block w takes part in entry j when bit 14 + w
-                    // is set.  Its S for an entry is issued one entry ahead, after its previous
-                    // PV (S_w and P_w share TMEM columns), its Q wait comes with its first S,
-                    // and its last S / PV release Q_w / hand O_w to the epilogue.
-                    const int4 meta = __ldg(p.bs_meta + bsparse_index(p, un.bh, un.i0));
-                    const uint16_t* lst = bsparse_list(p, un);
-                    const int n = meta.x;
-                    const int last[2] = {meta.y, meta.z};
-                    bool q_seen[2] = {false, false};
-                    bool pv_seen[2] = {false, false};
-                    int e_cur = __ldg(lst);
-                    int e_next = (n > 1) ? __ldg(lst + 1) : 0;
-                    if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int w = 0; w < 2; ++w) {
-                        if (!((e_cur >> (14 + w)) & 1)) continue;
-                        if (!(ok = wait(&bar_q[w], q_iter[w] & 1))) break;
-                        ++q_iter[w];
-                        q_seen[w] = true;
-                        tc_fence_after();
-                        issue_s(w, kc % S);
-                        if (last[w] == 0) umma_commit_w(&bar_q_free[w]);
-                    }
-                    if (!ok) break;
-                    umma_commit_w(&bar_kfree[kc % S]);
-                    for (int j = 0; ok && j < n; ++j) {
-                        const int e_after = (j + 2 < n) ? __ldg(lst + j + 2) : 0;  // in flight meanwhile
-                        const int s = (kc + j) % S;
-                        const int s1 = (kc + j + 1) % S;
-                        if (!(ok = wait(&bar_v[s], ((kc + j) / S) & 1))) break;
-                        bool k_ready = false;
-#pragma unroll
-                        for (int w = 0; w < 2; ++w) {
-                            if ((e_cur >> (14 + w)) & 1) {
-                                if (!pv_seen[w] && units_w[w] > 0) {
-                                    // O_w still holds the previous unit until its epilogue has read it
-                                    if (!(ok = wait(&bar_ofree[w], (units_w[w] - 1) & 1))) break;
-                                }
-                                if (!(ok = wait(&bar_p[2 * w], tp[w] & 1))) break;
-                                tc_fence_after();
-                                issue_pv_half(w, s, !pv_seen[w], 0);
-                                if (!(ok = wait(&bar_p[2 * w + 1], tp[w] & 1))) break;
-                                ++tp[w];
-                                tc_fence_after();
-                                issue_pv_half(w, s, !pv_seen[w], 1);
-                                pv_seen[w] = true;
-                                if (j == last[w]) {
-                                    umma_commit_w(&bar_o[w]);
-                                    ++units_w[w];
-                                }
-                            }
-                            if (j + 1 < n && ((e_next >> (14 + w)) & 1)) {
-                                if (!k_ready) {
-                                    if (!(ok = wait(&bar_k[s1], ((kc + j + 1) / S) & 1))) break;
-                                    tc_fence_after();
-                                    k_ready = true;
-                                }
-                                if (!q_seen[w]) {
-                                    if (!(ok = wait(&bar_q[w], q_iter[w] & 1))) break;
-                                    ++q_iter[w];
-                                    q_seen[w] = true;
-                                    tc_fence_after();
-                                }
-                                issue_s(w, s1);
-                                if (j + 1 == last[w]) umma_commit_w(&bar_q_free[w]);
-                            }
-                        }
-                        if (!ok) break;
-                        if (j + 1 < n) umma_commit_w(&bar_kfree[s1]);
-                        umma_commit_w(&bar_vfree[s]);
-                        e_cur = e_next;
-                        e_next = e_after;
-                    }
-                    kc += n;
-                    continue;
-                }
+                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, make_int4(0, 0, 0, 0));
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
@@ -565,8 +531,148 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 kc += n_max;
             }
             // Drain: every MMA issued by this thread completes before TMEM is freed.
-            umma_commit_w(bar_drain);
-            mbar_wait_drain(bar_drain, 0, p.status);
+            umma_commit_w(&bar_drain[0]);
+            mbar_wait_drain(&bar_drain[0], 0, p.status);
+        }
+    } else if (BSPARSE && (warp == 9 || warp == 10)) {
+        // ================= MMA issuers (block-sparse kernel): warp 9 for warpgroup 0, warp 10 for 1 ======
+        // Each issuer serves one softmax warpgroup, so neither waits on the other's
+        // softmax or epilogue; they meet only at the K/V ring, whose free barriers
+        // take one arrival from each.  The whole warp runs the loop, so descriptors
+        // and TMEM addresses are warp-uniform; one elected lane issues each MMA,
+        // commit and arrival (tcgen05.commit tracks the MMAs of the issuing thread).
+        const int w = warp - 9;
+        auto wait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, p.status));
+        };
+        auto arrive1 = [&](uint64_t* bar) {
+            if (lane == 0) mbar_arrive(bar);
+            __syncwarp();
+        };
+        {
+            constexpr uint32_t kIdescQK = idesc_bf16_f32(128, 128, 0, 0);
+            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
+            const uint32_t sQa = smem_u32(sQ) + w * Lay::kTileBytes, sKa = smem_u32(sK), sVa = smem_u32(sV);
+            const uint32_t t_s = tmem_base + w * 128;       // S_w, and P_w over it
+            const uint32_t t_o = tmem_base + 256 + w * D;   // O_w
+            // S_w = Q_w K_s^T into TMEM
+            auto issue_s = [&](int s) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * Lay::kBoxBytes + (kk & 3) * 32;
+                    const uint64_t a = smem_desc_sw128(sQa + koff, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(sKa + s * Lay::kTileBytes + koff, 16, 1024);
+                    umma_ss_w(t_s, a, b, kIdescQK, kk > 0 ? 1u : 0u);
+                }
+                umma_commit_w(&bar_s[w]);
+            };
+            // PV for one half of the tile's keys (h = 0: keys 0-63, h = 1: keys 64-127);
+            // the first PV of a unit overwrites O_w.
+            auto issue_pv_half = [&](int s, bool first, int h) {
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const int kk = h * 4 + k4;
+                    const uint64_t b =
+                        smem_desc_sw128(sVa + s * Lay::kTileBytes + kk * 2048, Lay::kBoxBytes, 1024);
+                    umma_ts_w(t_o, t_s + kk * 8, b, kIdescPV, (!first || kk > 0) ? 1u : 0u);
+                }
+            };
+            int kc = 0;        // ring position of the unit's first K/V tile
+            int q_iter = 0;    // Q_w tiles consumed
+            int tp = 0;        // P_w tiles consumed
+            int units_w = 0;   // units whose O_w was handed to the epilogue
+            bool ok = true;
+            for (int it = 0; ok; ++it) {
+                const int rs = it % kUnitRing;
+                if (!(ok = wait(&bar_ufull[rs], (it / kUnitRing) & 1))) break;
+                const int u = s_unit[rs];
+                const int4 meta = s_meta[rs];  // read before the slot is handed back
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_ufree[rs]);
+                if (u >= n_units) break;
+                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, meta);
+                // The unit's K/V tiles occupy ring positions kc .. kc + n_pos - 1; this
+                // warpgroup uses some of them (dense: the first n_w; block-sparse: the
+                // union-list entries with its bit), the last one at position `last`.
+                int n_pos, last;
+                const uint16_t* lst = nullptr;
+                ListWindow lw;
+                if constexpr (BSPARSE) {
+                    n_pos = meta.x;
+                    last = w == 0 ? meta.y : meta.z;
+                    lst = bsparse_list(p, un);
+                } else {
+                    n_pos = max(un.n_kv0, un.n_kv1);
+                    last = (w == 0 ? un.n_kv0 : un.n_kv1) - 1;
+                }
+                auto uses = [&](int j) -> bool {
+                    if constexpr (BSPARSE) return j <= last && ((lw.get(lst, j, n_pos) >> (14 + w)) & 1);
+                    else return j <= last;
+                };
+                // A position this warpgroup does not use still needs its arrivals on the
+                // free barriers; waiting for the tile's load first keeps each arrival in
+                // that position's phase (the load follows the previous phase of the slot).
+                auto skip = [&](int j) -> bool {
+                    const int pos = kc + j, s = pos % S;
+                    if (!wait(&bar_k[s], (pos / S) & 1)) return false;
+                    arrive1(&bar_kfree[s]);
+                    if (!wait(&bar_v[s], (pos / S) & 1)) return false;
+                    arrive1(&bar_vfree[s]);
+                    return true;
+                };
+                // S for used position j: Q_w comes with the unit's first S, and the last S
+                // of the unit releases Q_w to the producer.
+                bool q_seen = false;
+                auto issue_s_at = [&](int j) -> bool {
+                    const int pos = kc + j, s = pos % S;
+                    if (!wait(&bar_k[s], (pos / S) & 1)) return false;
+                    if (!q_seen) {
+                        if (!wait(&bar_q[w], q_iter & 1)) return false;
+                        ++q_iter;
+                        q_seen = true;
+                    }
+                    tc_fence_after();
+                    issue_s(s);
+                    umma_commit_w(&bar_kfree[s]);
+                    if (j == last) umma_commit_w(&bar_q_free[w]);
+                    return true;
+                };
+                int cur = 0;
+                while (ok && cur < n_pos && !uses(cur)) ok = skip(cur++);
+                if (ok && cur < n_pos) ok = issue_s_at(cur);
+                bool first_pv = true;
+                while (ok && cur < n_pos) {
+                    // PV for position cur (its S was issued), then the S of the next used
+                    // position: S_w and P_w share TMEM columns, and MMAs run in issue order.
+                    const int pos = kc + cur, s = pos % S;
+                    if (!(ok = wait(&bar_v[s], (pos / S) & 1))) break;
+                    if (first_pv && units_w > 0) {
+                        // O_w still holds the previous unit until its epilogue has read it
+                        if (!(ok = wait(&bar_ofree[w], (units_w - 1) & 1))) break;
+                    }
+                    if (!(ok = wait(&bar_p[2 * w], tp & 1))) break;
+                    tc_fence_after();
+                    issue_pv_half(s, first_pv, 0);
+                    if (!(ok = wait(&bar_p[2 * w + 1], tp & 1))) break;
+                    ++tp;
+                    tc_fence_after();
+                    issue_pv_half(s, first_pv, 1);
+                    first_pv = false;
+                    umma_commit_w(&bar_vfree[s]);
+                    if (cur == last) {
+                        umma_commit_w(&bar_o[w]);
+                        ++units_w;
+                    }
+                    int nxt = cur + 1;
+                    while (ok && nxt < n_pos && !uses(nxt)) ok = skip(nxt++);
+                    if (ok && nxt < n_pos) ok = issue_s_at(nxt);
+                    cur = nxt;
+                }
+                kc += n_pos;
+            }
+            // Drain: every MMA issued by this thread completes before TMEM is freed.
+            umma_commit_w(&bar_drain[w]);
+            mbar_wait_drain(&bar_drain[w], 0, p.status);
         }
     } else if (warp < 8) {
         // ================= softmax warpgroups =================
@@ -586,15 +692,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             ok = __all_sync(0xffffffffu, mbar_wait(&bar_ufull[rs], (it / kUnitRing) & 1, abort_flag, p.status));
             if (!ok) break;
             const int u = s_unit[rs];
+            int4 meta = make_int4(0, 0, 0, 0);
+            if constexpr (BSPARSE) meta = s_meta[rs];
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false);
+            const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, meta);
             int n = (w == 0) ? un.n_kv0 : un.n_kv1;
             const uint16_t* bs_own = nullptr;  // block-sparse: this query block's own list
             if constexpr (BSPARSE) {
                 const size_t ui = bsparse_index(p, un.bh, un.i0);
-                n = (__ldg(&p.bs_meta[ui].w) >> (16 * w)) & 0xffff;
+                n = (meta.w >> (16 * w)) & 0xffff;
                 bs_own = p.bs_own + (2 * ui + w) * p.bs_tk;
             }
             if (n == 0) continue;
