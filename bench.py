@@ -481,6 +481,25 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "frac_of_peak": round(fl / t_l / 1e12 / peaks["bf16_tflops"], 4), "launches": 1}
     del q, k, v, o, lse
 
+    # head dimension 256 (one 128-row Q tile per unit, 64-key K/V tiles)
+    w = WORKLOADS["fwd_d256_L4096"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+    o = torch.empty(B, H, L, d, dtype=torch.float32, device=device)
+    lse = torch.empty(B, H, L, dtype=torch.float32, device=device)
+
+    def fwd_d256():
+        rc = fa.fa_forward(q, k, v, o, lse, B, H, L, L, d, 1.0 / math.sqrt(d), 1, fa.FA_DT_F32, stream)
+        assert rc == fa.FA_OK
+
+    f256 = attn_flops(B, H, L, L, d, True)
+    t_256 = time_steps(fwd_d256, steps, warm, stream, dist, device) / steps
+    legs["fwd_d256_L4096"] = {"ms": round(t_256 * 1e3, 4), "TFLOP/s": round(f256 / t_256 / 1e12, 1),
+                              "frac_of_peak": round(f256 / t_256 / 1e12 / peaks["bf16_tflops"], 4), "launches": 1,
+                              "kernel": "fa_fwd256_kernel",
+                              "config": "B4 H16 L4096 d256 causal, O fp32 + LSE"}
+    del q, k, v, o, lse
+
     # decode over a 32,768-slot cache
     w = WORKLOADS["decode_cap32768"]
     B, H, cap, d = w["B"], w["H"], w["cap"], w["d"]

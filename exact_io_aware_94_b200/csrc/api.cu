@@ -258,14 +258,15 @@ const char* fa_status_string(int status) {
 int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,
                int d, float scale, int causal, int o_dtype, void* stream) {
     if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
     if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
         return FA_ERR_INVALID_ARG;
-    const long long n_ctas = static_cast<long long>(B) * H * ((Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta);
+    // units: 256 query rows (d <= 128) or 128 (d = 256) of one (b, h)
+    const long long n_ctas = static_cast<long long>(B) * H * ((Lq + 127) / 128);
     if (n_ctas > 0x7FFFFFFFLL) return FA_ERR_INVALID_ARG;
 
     DeviceState* st = nullptr;
@@ -274,9 +275,10 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
 
     FwdParams p{};
     const int BH = B * H;
+    const int kv_rows = d == 256 ? kFwd256BN : kFwdBN;  // keys per K/V tile
     if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, kFwdBM)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kv_rows)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kv_rows)) != FA_OK) return rc;
     if ((rc = encode_out_map_impl(&p.tm_o, o, BH, Lq, d, o_dtype)) != FA_OK) return rc;
     p.o = o;
     p.lse = lse;
@@ -290,7 +292,8 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
-    cudaError_t e = launch_fwd(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = d == 256 ? launch_fwd256(p, st->num_sms, static_cast<cudaStream_t>(stream))
+                             : launch_fwd(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -369,7 +372,7 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
 }
 
 size_t fa_decode_workspace_size(int B, int H, int cap, int d) {
-    if (B <= 0 || H <= 0 || cap <= 0 || (d != 64 && d != 128)) return 0;
+    if (B <= 0 || H <= 0 || cap <= 0 || (d != 64 && d != 128 && d != 256)) return 0;
     return decode_workspace_bytes(B, H, cap, d);
 }
 
@@ -377,7 +380,7 @@ int fa_decode(const void* q, const void* kcache, const void* vcache, const int* 
               int B, int H, int cap, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
               void* stream) {
     if (!q || !kcache || !vcache || !kv_lens || !o || !lse) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, cap, d) || !scale_ok(scale)) return FA_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(kcache, 16) || !aligned(vcache, 16) || !aligned(o, 16) ||
@@ -475,7 +478,7 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
 }
 
 size_t fa_decode_paged_workspace_size(int B, int H, int max_blocks, int page_size, int d) {
-    if (B <= 0 || H <= 0 || max_blocks <= 0 || page_size <= 0 || (d != 64 && d != 128)) return 0;
+    if (B <= 0 || H <= 0 || max_blocks <= 0 || page_size <= 0 || (d != 64 && d != 128 && d != 256)) return 0;
     const long long cap = static_cast<long long>(max_blocks) * page_size;
     if (cap > 0x7FFFFFFFLL) return 0;
     return decode_workspace_bytes(B, H, static_cast<int>(cap), d);
@@ -486,7 +489,7 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
                     int max_blocks, int d, float scale, int o_dtype, void* workspace, size_t workspace_bytes,
                     void* stream) {
     if (!q || !kpages || !vpages || !block_table || !kv_lens || !o || !lse) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (B <= 0 || H <= 0 || Hkv <= 0 || H % Hkv != 0 || num_pages <= 0 || max_blocks <= 0) return FA_ERR_INVALID_ARG;
     if (page_size <= 0 || page_size > 65536 || (page_size & (page_size - 1)) != 0) return FA_ERR_INVALID_ARG;

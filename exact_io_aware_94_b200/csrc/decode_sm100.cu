@@ -239,14 +239,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) fa_decode_split(DecodeParam
 // item is (b, KV head, group of GG query heads, chunk): every K and V row it
 // reads serves the whole group.  Warp 8 copies each 64-key stage of the item
 // (page segments of K and V, valid rows only) with 1-D bulk copies into a ring
-// of kPgStages stages.  In warps 0-7, D/8 lanes hold one key row slice (8 bf16)
+// of kPgStages<D> stages.  In warps 0-7, D/8 lanes hold one key row slice (8 bf16)
 // and keep, per head, a running max, a running sum and an 8-wide accumulator:
 // dot products and accumulation use packed FFMA2, and the accumulators are
 // rescaled only when a head's max grows by more than 2^8 (O = acc / l holds for
 // any common reference).  Bytes in flight are bounded by the ring (128 KB at
 // d = 128), not by registers.  Every wait is bounded; an abort drains the
 // copies in flight.
-constexpr int kPgStages = 4;
+// ring depth: 4 stages of 64 keys (128 KB of K and V at d = 128); 2 at d = 256
+template <int D>
+constexpr int kPgStages = (D == 256) ? 2 : 4;
 constexpr int kPgStageKeys = 64;
 constexpr int kPgThreads = 288;  // 8 compute warps + 1 copy warp
 
@@ -256,12 +258,12 @@ struct PagedTmaLayout {
     static constexpr int kGroups = 8 * (32 / kLanesPerKey);
     static constexpr int kStageBytes = kPgStageKeys * D * 2;  // one of K or V
     static constexpr int kKOff = 0;
-    static constexpr int kVOff = kKOff + kPgStages * kStageBytes;
-    static constexpr int kRedMOff = kVOff + kPgStages * kStageBytes;
+    static constexpr int kVOff = kKOff + kPgStages<D> * kStageBytes;
+    static constexpr int kRedMOff = kVOff + kPgStages<D> * kStageBytes;
     static constexpr int kRedLOff = kRedMOff + GG * kGroups * 4;
     static constexpr int kRedAccOff = kRedLOff + GG * kGroups * 4;
     static constexpr int kBarOff = (kRedAccOff + GG * kGroups * D * 4 + 7) / 8 * 8;
-    static constexpr int kMiscOff = kBarOff + 2 * kPgStages * 8;
+    static constexpr int kMiscOff = kBarOff + 2 * kPgStages<D> * 8;
     static constexpr int kBytes = kMiscOff + 16 + 128;
 };
 
@@ -284,12 +286,12 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
     float* red_l = reinterpret_cast<float*>(smem + Lay::kRedLOff);    // [GG][kGroups]
     float* red_acc = reinterpret_cast<float*>(smem + Lay::kRedAccOff);  // [GG][kGroups][D]
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
-    uint64_t* empty = full + kPgStages;
+    uint64_t* empty = full + kPgStages<D>;
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kPgStages; ++i) {
+        for (int i = 0; i < kPgStages<D>; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 8);
         }
@@ -332,9 +334,9 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
             const int end = min(start + kDecodeSplit, p.lens[b]);
             const int* table = p.block_table + static_cast<size_t>(b) * p.max_blocks;
             for (int k0 = start; k0 < end; k0 += kPgStageKeys, ++st) {
-                const int s = st % kPgStages;
-                if (st >= kPgStages) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / kPgStages) - 1) & 1, abort_flag, p.status));
+                const int s = st % kPgStages<D>;
+                if (st >= kPgStages<D>) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / kPgStages<D>) - 1) & 1, abort_flag, p.status));
                     if (!ok) break;
                 }
                 const int n = min(kPgStageKeys, end - k0);
@@ -367,8 +369,8 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
         }
         // every copy issued here lands before the CTA's shared memory goes away
         // (each barrier is at the phase of its last copy)
-        for (int t = max(0, st - kPgStages); t < st; ++t)
-            if (t != skipped) mbar_wait_drain(&full[t % kPgStages], (t / kPgStages) & 1, p.status);
+        for (int t = max(0, st - kPgStages<D>); t < st; ++t)
+            if (t != skipped) mbar_wait_drain(&full[t % kPgStages<D>], (t / kPgStages<D>) & 1, p.status);
     } else {
         // ---------------- compute warps 0-7
         const int g = warp * kGroupsPerWarp + lane / kLanesPerKey;
@@ -401,8 +403,8 @@ __global__ void __launch_bounds__(kPgThreads, 1) fa_decode_paged_tma(DecodeParam
                 for (int i = 0; i < 4; ++i) acc2[gg][i] = make_float2(0.0f, 0.0f);
             }
             for (int k0 = start; k0 < end; k0 += kPgStageKeys, ++st) {
-                const int s = st % kPgStages;
-                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (st / kPgStages) & 1, abort_flag, p.status));
+                const int s = st % kPgStages<D>;
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (st / kPgStages<D>) & 1, abort_flag, p.status));
                 if (!ok) break;
                 const int n = min(kPgStageKeys, end - k0);
                 float sc[kKeysPerGroup][GG];
@@ -565,6 +567,7 @@ cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaS
     fa_decode_plan<<<1, kPlanThreads, 0, stream>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (d == 256) return launch_paged_d<256>(p, num_sms, stream);
     return d == 128 ? launch_paged_d<128>(p, num_sms, stream) : launch_paged_d<64>(p, num_sms, stream);
 }
 
@@ -604,7 +607,11 @@ cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_
     if (e != cudaSuccess) return e;
     const long long upper = static_cast<long long>(p.B) * p.H * p.max_splits;
     const int grid = static_cast<int>(std::min<long long>(upper, static_cast<long long>(num_sms) * 3));
-    if (d == 128) {
+    if (d == 256) {
+        fa_decode_split<256><<<grid, kDecodeThreads, 0, stream>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        fa_decode_combine<256><<<p.B * p.H, 256, 0, stream>>>(p);
+    } else if (d == 128) {
         fa_decode_split<128><<<grid, kDecodeThreads, 0, stream>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         fa_decode_combine<128><<<p.B * p.H, 128, 0, stream>>>(p);

@@ -161,6 +161,9 @@ size_t bs_workspace_bytes(int B, int H, int Lq, int Lk);
 
 int fwd_smem_bytes(int d);
 cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
+// Head dimension 256: one 128-row Q tile per unit, K/V tiles of kFwd256BN keys.
+constexpr int kFwd256BN = 64;
+cudaError_t launch_fwd256(const FwdParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p, int d, int num_sms,
                                    cudaStream_t stream);

@@ -161,6 +161,8 @@ WORKLOADS = {
     "fwd_L4096_peaky": dict(kind="fwd", B=4, H=16, L=4096, d=128, causal=True, q_scale=4.0, seed=2),
     "train_L8192": dict(kind="fwdbwd", B=2, H=16, L=8192, d=128, causal=True, q_scale=1.0, seed=3),
     "long_L65536": dict(kind="fwd", B=1, H=8, L=65536, d=128, causal=True, q_scale=1.0, seed=4),
+    # Head dimension 256 at the 4,096-token shape.
+    "fwd_d256_L4096": dict(kind="fwd", B=4, H=16, L=4096, d=256, causal=True, q_scale=1.0, seed=9),
     "decode_cap32768": dict(kind="decode", B=64, H=32, cap=32768, d=128, len_lo=1024, len_hi=32768, seed=5),
     # Packed prefill batch of 16 causal sequences of 512 to 8,192 tokens.
     "prefill_varlen": dict(kind="varlen", B=16, H=16, d=128, len_lo=512, len_hi=8192, causal=True, seed=7),

@@ -70,7 +70,7 @@ extern "C" {
 typedef enum {
     FA_OK = 0,
     FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size or scale, misalignment, causal with Lq > Lk */
-    FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, dtype code unknown */
+    FA_ERR_UNSUPPORTED = 2, /* head dimension not supported by the call (see each call), dtype code unknown */
     FA_ERR_WORKSPACE = 3,   /* workspace pointer null or smaller than *_workspace_size() */
     FA_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
     FA_ERR_TIMEOUT = 5,     /* device: a bounded wait inside a kernel ran out */
@@ -88,8 +88,10 @@ enum { FA_DT_BF16 = 0, FA_DT_F32 = 1 };
  * Statistics").  Reads q [B,H,Lq,d], k and v [B,H,Lk,d] (bf16); writes
  * o [B,H,Lq,d] (bf16 if o_dtype == FA_DT_BF16, fp32 if FA_DT_F32) and
  * lse [B,H,Lq] (fp32).  scale multiplies q.k before the softmax (typically
- * 1/sqrt(d)).  d must be 64 or 128.  Rows never see keys beyond Lk; nothing
- * past the end of any tensor is read.
+ * 1/sqrt(d)).  d must be 64, 128 or 256 ("Basic Flash Attention Forward Pass"
+ * leaves D free; d = 256 runs a kernel with 128-row query tiles and 64-key K/V
+ * tiles).  Rows never see keys beyond Lk; nothing past the end of any tensor is
+ * read.
  */
 int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Lq, int Lk,
                int d, float scale, int causal, int o_dtype, void* stream);
@@ -151,7 +153,7 @@ size_t fa_decode_workspace_size(int B, int H, int cap, int d);
  * FlashAttention?", "What it changes for you": the cache lives in HBM and is
  * read once).  q [B,H,d] (bf16); kcache, vcache [B,H,cap,d] (bf16); kv_lens
  * int32 [B] on the device, the number of valid cache rows of each sequence.
- * Writes o [B,H,d] (o_dtype) and lse [B,H] (fp32).  Keys [0, kv_lens[b]) are
+ * Writes o [B,H,d] (o_dtype) and lse [B,H] (fp32).  d is 64, 128 or 256.  Keys [0, kv_lens[b]) are
  * split into fixed-size chunks processed in parallel; their partial
  * (O, LSE) pairs are merged by a log-sum-exp combine.  A length outside
  * [0, cap] is clamped and flagged as FA_ERR_KV_LEN in the status word; a
@@ -209,7 +211,7 @@ size_t fa_decode_paged_workspace_size(int B, int H, int max_blocks, int page_siz
  *   kv_lens     int32 [B] on the device, valid keys per sequence.
  *   o, lse      [B, H, d] (o_dtype) and [B, H] fp32.
  * Query head h reads KV head h / (H / Hkv).  H must be a multiple of Hkv and
- * page_size a power of two (1 .. 65536); d is 64 or 128.  q, kpages, vpages and
+ * page_size a power of two (1 .. 65536); d is 64, 128 or 256.  q, kpages, vpages and
  * o must be 16-byte aligned, the workspace 256-byte aligned (any torch
  * allocation is).  Lengths outside [0, max_blocks *
  * page_size] are clamped and flagged FA_ERR_KV_LEN; a table entry that a valid

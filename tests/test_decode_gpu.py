@@ -21,7 +21,7 @@ def poison_past_lengths(kc, vc, lens):
         vc[b, :, n:] = float("nan")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 def test_decode_small_with_edge_lengths(cuda_device, d):
     B, H, cap = 6, 3, 5000
     inp = decode_inputs(B, H, cap, d, seed=11 + d, len_lo=1, len_hi=cap)

@@ -41,6 +41,8 @@ def make_inputs(B, H, Hkv, ps, max_blocks, d, seed, lens):
     (128, 16, 2, 32, 80),   # groups of 8: two head groups per KV head
     (64, 6, 2, 1, 2600),    # groups of 3, one key per page
     (64, 8, 2, 128, 20),    # groups of 4 at d = 64
+    (256, 8, 2, 64, 40),    # groups of 4 at d = 256 (two-stage ring)
+    (256, 6, 3, 16, 160),   # groups of 2 at d = 256
 ])
 def test_decode_paged_parity_edge_lengths(cuda_device, d, H, Hkv, ps, max_blocks):
     cap = ps * max_blocks

@@ -44,6 +44,15 @@ SMALL = [
     (1, 1, 300, 100, 64, False, 1.0),     # Lq > Lk, non-causal
     (1, 1, 257, 513, 64, True, 4.0),
     (2, 1, 600, 600, 128, True, 8.0),     # very peaky rows
+    # head dimension 256 (one 128-row Q tile per unit, 64-key tiles)
+    (1, 1, 1, 1, 256, True, 1.0),
+    (1, 2, 63, 63, 256, False, 1.0),
+    (2, 2, 200, 200, 256, True, 1.0),
+    (1, 1, 384, 384, 256, True, 4.0),
+    (1, 2, 700, 700, 256, False, 1.0),
+    (1, 1, 100, 321, 256, True, 1.0),     # Lq < Lk: bottom-right causal alignment
+    (1, 1, 300, 65, 256, False, 1.0),     # Lq > Lk, non-causal
+    (1, 1, 520, 520, 256, True, 8.0),     # very peaky rows: rescaling in the split rows
 ]
 
 
