@@ -498,7 +498,24 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                               "frac_of_peak": round(f256 / t_256 / 1e12 / peaks["bf16_tflops"], 4), "launches": 1,
                               "kernel": "fa_fwd256_kernel",
                               "config": "B4 H16 L4096 d256 causal, O fp32 + LSE"}
-    del q, k, v, o, lse
+    g256 = torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), device)
+
+    def bwd_d256():
+        rc = fa.fa_backward(q, k, v, o, g256, lse, dq, dk, dv, B, H, L, L, d, 1.0 / math.sqrt(d), 1, fa.FA_DT_F32,
+                            ws, ws.numel(), stream)
+        assert rc == fa.FA_OK
+
+    fb256 = attn_flops(B, H, L, L, d, True, backward=True)
+    t_b256 = time_steps(bwd_d256, steps, warm, stream, dist, device) / steps
+    legs["bwd_d256_L4096"] = {"ms": round(t_b256 * 1e3, 4), "TFLOP/s": round(fb256 / t_b256 / 1e12, 1),
+                              "frac_of_peak": round(fb256 / t_b256 / 1e12 / peaks["bf16_tflops"], 4),
+                              "launches": 3, "kernels": "fa_bwd_dot + fa_bwd_dkdv256 + fa_bwd_dq256",
+                              "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 9 (dK/dV halves "
+                                                  "recompute S^T and dP^T; dQ recomputes S and dP)",
+                              "config": "B4 H16 L4096 d256 causal"}
+    del q, k, v, o, lse, g256, dq, dk, dv, ws
 
     # decode over a 32,768-slot cache
     w = WORKLOADS["decode_cap32768"]

@@ -181,7 +181,7 @@ int bwd_check_args(const void* q, const void* k, const void* v, const void* o, c
                    const void* dq, const void* dk, const void* dv, int B, int H, int Lq, int Lk, int d, float scale,
                    int causal, int o_dtype) {
     if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
@@ -190,7 +190,7 @@ int bwd_check_args(const void* q, const void* k, const void* v, const void* o, c
         !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
         return FA_ERR_INVALID_ARG;
     const long long bh = static_cast<long long>(B) * H;
-    if (bh * ((Lq + 127) / 128) > 0x7FFFFFFFLL || bh * ((Lk + 127) / 128) > 0x7FFFFFFFLL ||
+    if (bh * ((Lq + 127) / 128) > 0x7FFFFFFFLL || bh * ((Lk + 127) / 128) * 2 > 0x7FFFFFFFLL ||
         bh * Lq * (d / 8) / 256 > 0x7FFFFFFFLL)
         return FA_ERR_INVALID_ARG;
     return FA_OK;
@@ -209,6 +209,12 @@ int bwd_launch_checked(const void* q, const void* k, const void* v, const void* 
     if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, 128)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, 128)) != FA_OK) return rc;
     if ((rc = encode_rows_map(&p.tm_do, dO, BH, Lq, d, 128)) != FA_OK) return rc;
+    if (d == 256) {
+        if ((rc = encode_rows_map(&p.tm_q64, q, BH, Lq, d, 64)) != FA_OK) return rc;
+        if ((rc = encode_rows_map(&p.tm_k64, k, BH, Lk, d, 64)) != FA_OK) return rc;
+        if ((rc = encode_rows_map(&p.tm_v64, v, BH, Lk, d, 64)) != FA_OK) return rc;
+        if ((rc = encode_rows_map(&p.tm_do64, dO, BH, Lq, d, 64)) != FA_OK) return rc;
+    }
     p.o = o;
     p.dO = dO;
     p.lse = lse;
@@ -415,7 +421,7 @@ int fa_decode(const void* q, const void* kcache, const void* vcache, const int* 
 }
 
 size_t fa_backward_workspace_size(int B, int H, int Lq, int Lk, int d) {
-    if (B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || (d != 64 && d != 128)) return 0;
+    if (B <= 0 || H <= 0 || Lq <= 0 || Lk <= 0 || (d != 64 && d != 128 && d != 256)) return 0;
     return bwd_workspace_bytes(B, H, Lq);
 }
 

@@ -717,6 +717,12 @@ size_t bwd_workspace_bytes(int B, int H, int Lq) {
 }
 
 cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream) {
+    if (d == 256) {
+        const long long threads = static_cast<long long>(p.B) * p.H * p.Lq * (256 / 8);
+        fa_bwd_dot<256><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(p);
+        const cudaError_t e = cudaGetLastError();
+        return e != cudaSuccess ? e : launch_bwd256_main(p, stream);
+    }
     return d == 128 ? launch_bwd_d<128>(p, stream) : launch_bwd_d<64>(p, stream);
 }
 

@@ -82,6 +82,9 @@ struct __align__(64) BwdParams {
     CUtensorMap tm_k;   // [B*H, Lk, d]
     CUtensorMap tm_v;   // [B*H, Lk, d]
     CUtensorMap tm_do;  // [B*H, Lq, d]
+    // d = 256 only: the same tensors with 64-row boxes (64-query tiles of the dK/dV
+    // kernel, 64-key tiles of the dQ kernel)
+    CUtensorMap tm_q64, tm_k64, tm_v64, tm_do64;
     const void* o;      // forward output, o_dtype
     const void* dO;     // bf16 [B, H, Lq, d]
     const float* lse;   // [B, H, Lq]
@@ -113,6 +116,7 @@ bool shape_ok(int B, int H, int L, int d);
 // right for a positive, finite scale (zero would turn -inf * 0 into NaN).
 inline bool scale_ok(float scale) { return scale > 0.0f && scale <= 3.4028234663852886e38f; }
 cudaError_t launch_bwd(const BwdParams& p, int d, cudaStream_t stream);
+cudaError_t launch_bwd256_main(const BwdParams& p, cudaStream_t stream);
 
 // Decode: keys of each sequence are cut into chunks of kDecodeSplit keys.
 constexpr int kDecodeSplit = 1024;

@@ -33,6 +33,13 @@ SMALL = [
     (1, 1, 300, 100, 64, False),
     (1, 1, 200, 333, 64, True),
     (2, 1, 520, 520, 128, True),
+    # head dimension 256 (dK/dV by halves of d, 64-query and 64-key tiles)
+    (1, 1, 3, 3, 256, True),       # (a single key gives dQ = 0 exactly: no relative error to grade)
+    (1, 2, 70, 70, 256, True),
+    (2, 1, 200, 200, 256, False),
+    (1, 1, 100, 300, 256, True),   # bottom-right causal
+    (1, 1, 300, 130, 256, False),
+    (1, 2, 384, 384, 256, True),
 ]
 
 
@@ -95,3 +102,13 @@ def test_backward_full_size_sampled_heads(cuda_device):
     dv_sum = dv.double().sum(dim=2).cpu().numpy()
     g_sum = inp.dO.double().sum(dim=2).numpy()
     assert rel_fro(dv_sum, g_sum) < 1e-2
+
+
+def test_backward_d256_determinism(cuda_device):
+    """d = 256: two runs give bitwise identical gradients (no atomics)."""
+    inp = attention_inputs(1, 2, 333, 333, 256, seed=19, with_dO=True)
+    scale = 1.0 / 16.0
+    a = gpu_fwd_bwd(inp, scale, True, cuda_device)
+    b = gpu_fwd_bwd(inp, scale, True, cuda_device)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
