@@ -654,6 +654,7 @@ def run_profile_case(args, device):
     bwd: forward then backward at the 8,192-token training shape; decode_small:
     decode at B=16 H=32 cap=8192 (1 GiB of cache, small enough to capture);
     varlen_small: packed causal forward of 8 sequences of 512..4,096 tokens;
+    fwd256: the d = 256 forward at B=4 H=16 L=4,096;
     decode_paged_small: paged, grouped-head decode at B=16 H=32 Hkv=8;
     blocksparse_small: block-sparse causal forward at B=2 H=16 L=8192 with the
     benchmark's mask recipe (192 MiB of Q/K/V, more than L2)."""
@@ -678,6 +679,15 @@ def run_profile_case(args, device):
             ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), device)
             for _ in range(calls):
                 fa.backward(q, k, v, o, g, lse, causal=True, ws=ws, stream=stream)
+        nbytes = 0
+    elif args.profile_case == "fwd256":
+        # head dimension 256: the d = 256 forward at B4 H16 L4096 causal (384 MiB of Q/K/V)
+        w = WORKLOADS["fwd_d256_L4096"]
+        B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+        q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
+        o, lse = fa.forward(q, k, v, causal=True, stream=stream)
+        for _ in range(calls):
+            fa.forward(q, k, v, causal=True, out=o, lse=lse, stream=stream)
         nbytes = 0
     elif args.profile_case == "varlen_small":
         # 8 causal sequences of 512..4,096 tokens, H16 d128 (about 1 GB on the device)
@@ -777,7 +787,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
     ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small", "varlen_small", "decode_paged_small",
-                                                    "blocksparse_small"],
+                                                    "blocksparse_small", "fwd256"],
                     default=None,
                     help="run only this path W+K times for a profiler; no benchmark line")
     args = ap.parse_args(argv)

@@ -231,6 +231,8 @@ int bwd_launch_checked(const void* q, const void* k, const void* v, const void* 
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
+    p.hg_kv = heads_per_l2_group(2LL * Lq * d * 2, BH);
+    p.hg_q = heads_per_l2_group(2LL * Lk * d * 2, BH);
     const cudaError_t e = launch_bwd(p, d, stream);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -298,6 +300,7 @@ int fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
+    p.head_group = heads_per_l2_group(2LL * Lk * d * 2, BH);
     cudaError_t e = d == 256 ? launch_fwd256(p, st->num_sms, static_cast<cudaStream_t>(stream))
                              : launch_fwd(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -373,6 +376,7 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = plan.causal;
     p.o_dtype = o_dtype;
+    p.head_group = heads_per_l2_group(2LL * Lk * d * 2, BH);
     cudaError_t e = launch_fwd_blocksparse(plan, p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -79,9 +79,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int BH = p.B * p.H;
     const int half = static_cast<int>(blockIdx.x) & 1;   // columns [128 half, 128 half + 128) of dK, dV
-    const int tile = static_cast<int>(blockIdx.x) >> 1;
-    const int kt = tile / BH;  // small key tiles first: they see the most queries
-    const int bh = tile % BH;
+    // small key tiles first (they see the most queries), in groups of heads whose Q and dO stay in L2
+    int kt, bh;
+    grouped_block(static_cast<int>(blockIdx.x) >> 1, BH, (p.Lk + 127) / 128, p.hg_kv, kt, bh);
     const int j0 = kt * 128;
     const int off = p.Lk - p.Lq;
     const int nq_all = (p.Lq + 63) / 64;
@@ -357,8 +357,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int BH = p.B * p.H;
     const int nq_all = (p.Lq + 127) / 128;
-    const int qt = nq_all - 1 - static_cast<int>(blockIdx.x) / BH;  // long causal rows first
-    const int bh = static_cast<int>(blockIdx.x) % BH;
+    // long causal rows first, in groups of heads whose K and V stay in L2
+    int t, bh;
+    grouped_block(static_cast<int>(blockIdx.x), BH, nq_all, p.hg_q, t, bh);
+    const int qt = nq_all - 1 - t;
     const int i0 = qt * 128;
     const int off = p.Lk - p.Lq;
     const int nk_all = (p.Lk + 63) / 64;

@@ -75,7 +75,21 @@ struct __align__(64) FwdParams {
     float scale_log2;  // scale * log2(e)
     int causal;
     int o_dtype;
+    int head_group;    // batched and block-sparse kernels: heads per group of the unit order (>= 1)
 };
+
+// Heads whose K and V (or, for the backward, whose re-read tensors) are kept in
+// L2 together by the unit and block orders: bytes_per_head of the re-read data
+// against a budget of about a quarter of the 126 MB L2.  When not even two heads
+// fit, the heads are not grouped at all (one group of all of them): with many
+// CTAs on each long head, interleaving the heads measured faster than taking
+// them one at a time.
+inline int heads_per_l2_group(long long bytes_per_head, int BH) {
+    const long long budget = 32LL << 20;
+    long long g = bytes_per_head > 0 ? budget / bytes_per_head : BH;
+    if (g < 2 || g > BH) g = BH;
+    return static_cast<int>(g);
+}
 
 struct __align__(64) BwdParams {
     CUtensorMap tm_q;   // [B*H, Lq, d] bf16, box {64, 128, 1}
@@ -97,7 +111,20 @@ struct __align__(64) BwdParams {
     float scale, scale_log2;
     int causal;
     int o_dtype;
+    // block orders: heads per group whose Q and dO (dK/dV kernels) or K and V (dQ
+    // kernels) stay in L2 together (>= 1)
+    int hg_kv, hg_q;
 };
+
+// Block b of a grid of BH * n tiles, in groups of G heads: within a group, tile
+// index t = 0, 1, ... slowest, heads interleaved.  Returns (t, bh).
+__device__ __forceinline__ void grouped_block(int b, int BH, int n, int G, int& t, int& bh) {
+    const int grp = b / (G * n);
+    const int r = b - grp * G * n;
+    const int gsz = min(G, BH - grp * G);
+    t = r / gsz;
+    bh = grp * G + r % gsz;
+}
 
 size_t bwd_workspace_bytes(int B, int H, int Lq);
 

@@ -68,14 +68,19 @@ struct Unit256 {
     int bh, i0, n;  // (b*H + h), first query row, 64-key tiles to visit
 };
 
-// Units in a fixed global order: longest causal rows first (query tile index
-// descending), heads interleaved.
+// Units in a fixed global order: the (b, h) pairs in groups of p.head_group heads
+// whose K and V fit in L2 together; within a group, longest causal rows first
+// (query tile index descending), heads interleaved.
 __device__ __forceinline__ Unit256 unit256_of(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
     const int n_qt = (p.Lq + kBM - 1) / kBM;
+    const int G = p.head_group;
+    const int grp = u / (G * n_qt);
+    const int rem = u - grp * G * n_qt;
+    const int gsz = min(G, BH - grp * G);
     Unit256 r;
-    const int qt = n_qt - 1 - u / BH;
-    r.bh = u % BH;
+    const int qt = n_qt - 1 - rem / gsz;
+    r.bh = grp * G + rem % gsz;
     r.i0 = qt * kBM;
     const int n_all = (p.Lk + kBN - 1) / kBN;
     if (p.causal) {

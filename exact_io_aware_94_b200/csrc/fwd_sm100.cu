@@ -95,14 +95,26 @@ struct Unit {
     int q0, k0, lq, lk;
 };
 
-// Units in a fixed global order: longest causal rows first (pair index
-// descending), heads interleaved.
-__device__ __forceinline__ Unit unit_of(const FwdParams& p, int u) {
+// Units in a fixed global order: the (b, h) pairs are taken in groups of
+// p.head_group heads whose K and V fit in L2 together; within a group, longest
+// causal rows first (pair index descending), heads interleaved.  At any time the
+// CTAs then read the K/V of about one group, which stays in L2, and the last
+// units of the launch are still the shortest.
+__device__ __forceinline__ void unit_pair_head(const FwdParams& p, int u, int n_pairs, int& pair, int& bh) {
     const int BH = p.B * p.H;
+    const int G = p.head_group;
+    const int grp = u / (G * n_pairs);
+    const int r = u - grp * G * n_pairs;
+    const int gsz = min(G, BH - grp * G);  // heads in this group (the last one may be short)
+    pair = n_pairs - 1 - r / gsz;
+    bh = grp * G + r % gsz;
+}
+
+__device__ __forceinline__ Unit unit_of(const FwdParams& p, int u) {
     const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
     Unit r;
-    const int pair = n_pairs - 1 - u / BH;
-    r.bh = u % BH;
+    int pair;
+    unit_pair_head(p, u, n_pairs, pair, r.bh);
     r.i0 = pair * kFwdRowsPerCta;
     const int n_kv_all = (p.Lk + kFwdBN - 1) / kFwdBN;
     const int off = p.Lk - p.Lq;  // causal: query i sits at key position i + off
@@ -178,11 +190,10 @@ __device__ __forceinline__ size_t bsparse_index(const FwdParams& p, int bh, int 
 
 // meta: the unit's bs_meta entry (its first field is the union-list length).
 __device__ __forceinline__ Unit unit_of_bsparse(const FwdParams& p, int u, const int4& meta) {
-    const int BH = p.B * p.H;
     const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
     Unit r;
-    const int pair = n_pairs - 1 - u / BH;
-    r.bh = u % BH;
+    int pair;
+    unit_pair_head(p, u, n_pairs, pair, r.bh);
     r.i0 = pair * kFwdRowsPerCta;
     const int cnt = meta.x;
     r.n_kv0 = cnt;
@@ -210,9 +221,10 @@ __device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag, c
 
 // The block-sparse metadata of unit u (read by the producer only).
 __device__ __forceinline__ int4 bsparse_meta_of(const FwdParams& p, int u) {
-    const int BH = p.B * p.H;
     const int n_pairs = (p.Lq + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
-    return __ldg(p.bs_meta + bsparse_index(p, u % BH, (n_pairs - 1 - u / BH) * kFwdRowsPerCta));
+    int pair, bh;
+    unit_pair_head(p, u, n_pairs, pair, bh);
+    return __ldg(p.bs_meta + bsparse_index(p, bh, pair * kFwdRowsPerCta));
 }
 
 // Entry j of a unit's key-block list, read 32 entries at a time by the whole
