@@ -75,6 +75,17 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Source files whose state a recorded ncu capture of each kernel family depends on:
+# the kernel file, the PTX helpers, the shared internal header and the host API
+# (tile maps, unit orders and launch shapes are set there).
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ["fwd_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+    "fa_fwd256_kernel": ["fwd256_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+    "fa_bwd": ["bwd_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+    "fa_decode": ["decode_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+}
+
+
 def kernel_source_hash(files):
     h = hashlib.sha256()
     for f in files:
@@ -83,8 +94,11 @@ def kernel_source_hash(files):
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel, workload, src_files):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged since."""
+def recorded_traffic(kernel, workload, algorithmic_bytes=None):
+    """DRAM bytes (read + write) per launch from a committed ncu summary, if the
+    kernel's sources are unchanged since the capture.  A record taken on a smaller
+    case of the same kernel stores its traffic/algorithmic ratio instead, which is
+    applied to this workload's algorithmic bytes."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as fh:
@@ -92,9 +106,13 @@ def recorded_traffic(kernel, workload, src_files):
     except (OSError, ValueError):
         return None
     e = rec.get(kernel, {}).get(workload)
-    if not e or e.get("source_hash") != kernel_source_hash(src_files):
+    if not e or e.get("source_hash") != kernel_source_hash(KERNEL_SOURCES[kernel]):
         return None
-    return e.get("bytes_per_launch")
+    if "bytes_per_launch" in e:
+        return e["bytes_per_launch"]
+    if "traffic_over_algorithmic" in e and algorithmic_bytes:
+        return int(round(e["traffic_over_algorithmic"] * algorithmic_bytes))
+    return None
 
 
 def reduce_max(value, dist=None, device=None):
@@ -318,7 +336,7 @@ def run_ours(args, dist, rank, world, device):
             "peak": peaks["bf16_tflops"], "peak_kind": peak_kind + " burst bf16 (cuBLAS 8192^3)",
             "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
             "frac_of_nominal_2250": round(achieved / NOMINAL_BF16_TFLOPS, 4),
-            "traffic": recorded_traffic("fa_fwd_kernel", HEADLINE, ["fwd_sm100.cu", "ptx.cuh"]),
+            "traffic": recorded_traffic("fa_fwd_kernel", HEADLINE),
             "algorithmic_flops_per_launch": flops}
 
     # ---- end to end through the public API: every step copies its Q/K/V in from pinned host
@@ -461,7 +479,7 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "frac_of_peak": round(fb / t_b / 1e12 / peaks["bf16_tflops"], 4),
                                "launches": 3, "kernels": "fa_bwd_dot + fa_bwd_dkdv + fa_bwd_dq",
                                "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 7",
-                               "traffic": recorded_traffic("fa_bwd", "train_L8192", ["bwd_sm100.cu", "ptx.cuh"])}
+                               "traffic": recorded_traffic("fa_bwd", "train_L8192")}
     del q, k, v, g, o, lse, dq, dk, dv, ws
 
     # 65,536-token forward
@@ -497,6 +515,7 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
     legs["fwd_d256_L4096"] = {"ms": round(t_256 * 1e3, 4), "TFLOP/s": round(f256 / t_256 / 1e12, 1),
                               "frac_of_peak": round(f256 / t_256 / 1e12 / peaks["bf16_tflops"], 4), "launches": 1,
                               "kernel": "fa_fwd256_kernel",
+                              "traffic": recorded_traffic("fa_fwd256_kernel", "fwd_d256_L4096"),
                               "config": "B4 H16 L4096 d256 causal, O fp32 + LSE"}
     g256 = torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -542,7 +561,7 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                "frac_of_nominal_8000": round(nbytes / t_d / 1e9 / NOMINAL_HBM_GBS, 4),
                                "launches": 3, "kernels": "fa_decode_plan + fa_decode_split + fa_decode_combine",
                                "l2": "caches 2 x 16 GiB, far larger than L2",
-                               "traffic": recorded_traffic("fa_decode", "decode_cap32768", ["decode_sm100.cu"])}
+                               "traffic": recorded_traffic("fa_decode", "decode_cap32768", nbytes)}
     del kc, vc
 
     # packed prefill batch of sequences of different lengths (causal)
@@ -599,6 +618,7 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                    "frac_of_peak": round(fs / t_s / 1e12 / peaks["bf16_tflops"], 4),
                                    "launches": 2, "kernels": "fa_bsparse_plan + fa_fwd_kernel (block-sparse)",
                                    "permitted_fraction_of_causal": round(density, 4),
+                                   "traffic": recorded_traffic("fa_fwd_kernel", "prefill_blocksparse"),
                                    "config": "B2 H16 L16384 d128 causal; per-head block mask: sink block, window "
                                              "of 8 key blocks, 10% of other blocks below the diagonal; TFLOP/s "
                                              "counts permitted pairs only"}
@@ -637,7 +657,8 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                 "frac_of_peak": round(nbytes / t_p / 1e9 / peaks["hbm_gbs"], 4),
                                 "frac_of_nominal_8000": round(nbytes / t_p / 1e9 / NOMINAL_HBM_GBS, 4),
                                 "launches": 3,
-                                "kernels": "fa_decode_plan + fa_decode_paged_split + fa_decode_combine",
+                                "kernels": "fa_decode_plan + fa_decode_paged_tma + fa_decode_combine",
+                                "traffic": recorded_traffic("fa_decode", "decode_paged_gqa", nbytes),
                                 "config": "B64 H32 Hkv8 (groups of 4) d128, 64-token pages in shuffled order, "
                                           "lengths U[1024, 32768]",
                                 "l2": "pages 2 x %.1f GiB, far larger than L2" % (kp.numel() * 2 / 2 ** 30)}
