@@ -115,6 +115,19 @@ int encode_rows_map(CUtensorMap* map, const void* base, int BH, int L, int d, in
     return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// A paged K or V pool [rows][d] bf16 (rows = num_pages * Hkv * page_size) as a
+// 2-D map with boxes of 64 columns x box_rows rows and 128-byte swizzle.
+int encode_pool_map(CUtensorMap* map, const void* base, long long rows, int d, int box_rows) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // O written by TMA stores: [BH, L, d] in fp32 or bf16, boxes of 32 rows x
 // 128 bytes (32 fp32 or 64 bf16 columns), 128-byte swizzle.  Rows past L are
 // clipped by the copy engine.
@@ -540,6 +553,16 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
     while ((1 << shift) < page_size) ++shift;
     p.page_shift = shift;
     p.max_blocks = max_blocks;
+    // the tensor-core kernel needs boxes of at least 8 rows (one 1,024-byte swizzle atom)
+    // and pool row indices that fit the map's int32 coordinates
+    const long long pool_rows = static_cast<long long>(num_pages) * Hkv * page_size;
+    p.pool_box_rows = 0;
+    if ((d == 64 || d == 128) && page_size >= 8 && pool_rows <= 0x7FFFFFFFLL) {
+        const int br = page_size < 64 ? page_size : 64;
+        if ((rc = encode_pool_map(&p.tm_kpool, kpages, pool_rows, d, br)) != FA_OK) return rc;
+        if ((rc = encode_pool_map(&p.tm_vpool, vpages, pool_rows, d, br)) != FA_OK) return rc;
+        p.pool_box_rows = br;
+    }
     decode_carve_workspace(p, workspace, B, H, static_cast<int>(cap), d);
     cudaError_t e = launch_decode_paged(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -563,7 +586,8 @@ int fa_check_status(void* stream) {
 #ifdef FA_TEST_HOOKS
 // Fault injection for the tests of the bounded waits; exported by the test build
 // (libfa_sm100_testhooks.so) only.  where: 1 = forward K tile, 2 = dK/dV K/V
-// tiles, 3 = paged-decode stage.  Arms a one-shot fault on the current device.
+// tiles, 3 = paged-decode stage (d <= 128), 4 = paged-decode stage (d = 256).
+// Arms a one-shot fault on the current device.
 int fa_test_inject_fault(int where) {
     DeviceState* st = nullptr;
     const int rc = device_state(&st);
@@ -571,7 +595,8 @@ int fa_test_inject_fault(int where) {
     cudaError_t e = cudaErrorInvalidValue;
     if (where == 1) e = fwd_test_arm_skip_k();
     else if (where == 2) e = bwd_test_arm_skip_kv();
-    else if (where == 3) e = paged_test_arm_skip_stage();
+    else if (where == 3) e = paged_mma_test_arm_skip_stage();
+    else if (where == 4) e = paged_test_arm_skip_stage();
     else return FA_ERR_INVALID_ARG;
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -39,9 +39,9 @@ namespace {
 constexpr int kPlanThreads = 1024;
 
 #ifdef FA_TEST_HOOKS
-// One-shot fault (test build only): the next stage a paged-decode copy warp
-// would fill gets neither its expected byte count nor its copies, so the
-// compute warps' wait for it runs out.
+// One-shot fault (test build only): the next stage a paged-decode copy warp of
+// the d = 256 kernel would fill gets neither its expected byte count nor its
+// copies, so the compute warps' wait for it runs out.
 __device__ int g_test_skip_stage;
 #endif
 
@@ -549,11 +549,14 @@ cudaError_t launch_paged_tma(const DecodeParams& p, int num_sms, cudaStream_t st
     return cudaGetLastError();
 }
 
+// d = 64, 128 with pages of at least 8 rows: the tensor-core split kernel
+// (decode_paged_mma.cu); otherwise the CUDA-core split kernel above.
 template <int D>
 cudaError_t launch_paged_d(const DecodeParams& p, int num_sms, cudaStream_t stream) {
     const int group = p.H / p.Hkv;
     cudaError_t e;
-    if (group % 4 == 0) e = launch_paged_tma<D, 4>(p, num_sms, stream);
+    if (D != 256 && p.pool_box_rows > 0) e = launch_paged_mma_split(p, D, num_sms, stream);
+    else if (group % 4 == 0) e = launch_paged_tma<D, 4>(p, num_sms, stream);
     else if (group % 2 == 0) e = launch_paged_tma<D, 2>(p, num_sms, stream);
     else e = launch_paged_tma<D, 1>(p, num_sms, stream);
     if (e != cudaSuccess) return e;

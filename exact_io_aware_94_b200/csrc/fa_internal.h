@@ -24,7 +24,8 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 // producer.  Each returns a CUDA error code.
 cudaError_t fwd_test_arm_skip_k();      // forward: the next K tile a producer would load is never loaded
 cudaError_t bwd_test_arm_skip_kv();     // dK/dV kernel: the next CTA's K/V tiles are never loaded
-cudaError_t paged_test_arm_skip_stage();  // paged decode: the next stage's copies are never issued
+cudaError_t paged_test_arm_skip_stage();  // paged decode, d = 256: the next stage's copies are never issued
+cudaError_t paged_mma_test_arm_skip_stage();  // paged decode, d <= 128: the same
 #endif
 
 // Forward kernel tiling: two 128-row Q tiles per CTA (one per softmax
@@ -149,7 +150,12 @@ cudaError_t launch_bwd256_main(const BwdParams& p, cudaStream_t stream);
 constexpr int kDecodeSplit = 1024;
 constexpr int kDecodeThreads = 256;
 
-struct DecodeParams {
+struct __align__(64) DecodeParams {
+    // paged cache on the tensor cores (d = 64, 128, page_size >= 8): the K and V page pools as
+    // 2-D maps [num_pages * Hkv * page_size rows][d], boxes of 64 columns x pool_box_rows rows
+    // (min(page_size, 64)), 128-byte swizzle.  pool_box_rows = 0: the CUDA-core kernel instead.
+    CUtensorMap tm_kpool, tm_vpool;
+    int pool_box_rows;
     const void* q;        // [B, H, d] bf16
     const void* k;        // [B, H, cap, d] bf16
     const void* v;        // [B, H, cap, d] bf16
@@ -174,6 +180,9 @@ size_t decode_workspace_bytes(int B, int H, int cap, int d);
 void decode_carve_workspace(DecodeParams& p, void* ws, int B, int H, int cap, int d);
 cudaError_t launch_decode(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode_paged(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
+// The split step of the paged decode at d = 64, 128 on the tensor cores (the
+// combine is launched by launch_decode_paged).
+cudaError_t launch_paged_mma_split(const DecodeParams& p, int d, int num_sms, cudaStream_t stream);
 
 // Block-sparse planning: per 256-row unit, the key blocks (after the causal cut)
 // that either of its two 128-row query blocks may see, in increasing order.
