@@ -834,18 +834,68 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             if (!ok) break;
             ++nunits;
             tc_fence_after();
+            // fp32 O of the batched and block-sparse kernels is stored directly from
+            // registers; for that, O is read with the 16x256b shape: four consecutive
+            // threads then hold 32 contiguous bytes of one row, so each store instruction
+            // writes whole 32-byte sectors (eight rows x 32 bytes), with no staging and
+            // no wait on the copy engine.  Other outputs go through the TMA-store path.
+            const bool direct = !VARLEN && p.o_dtype == FA_DT_F32;
             uint32_t ov[D];
+            if (direct) {
+                // ov[(16h + c/8... ) ]: half h = lanes [16h, 16h + 16) of the warp, 64-column block b
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld32(t_o + c * 32, r);
+                for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) ov[c * 32 + x] = r[x];
+                    for (int b = 0; b < D / 64; ++b) {
+                        uint32_t r[32];
+                        tmem_ld_16x256b_x8(t_o + (static_cast<uint32_t>(16 * h) << 16) + b * 64, r);
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) ov[(h * (D / 64) + b) * 32 + x] = r[x];
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(t_o + c * 32, r);
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) ov[c * 32 + x] = r[x];
+                }
             }
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bar_ofree[w]);  // O_w may now be overwritten by the next unit's PV
-            {
+            if (direct) {
+                // Rows held by this thread: rsub + 8k of the warp's 32 (k = 0..3: half h = k / 2,
+                // upper 8 rows of the half when k is odd); their normalisers come from the
+                // threads that own those rows.  Block-sparse rows that see no key store 0.
+                const float den = l + corr;
+                const bool empty_row = BSPARSE && !(den > 0.0f);
+                const float inv_l = empty_row ? 0.0f : 1.0f / den;
+                const int rsub = lane >> 2, cp = (lane & 3) * 2;
+                float* obase = static_cast<float*>(p.o) +
+                               (static_cast<size_t>(un.bh) * p.Lq + tile_first_row + wq * 32) * D;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int rl = rsub + 8 * k;  // row within the warp's 32
+                    const float inv = __shfl_sync(0xffffffffu, inv_l, rl);
+                    const bool zero = __shfl_sync(0xffffffffu, empty_row ? 1 : 0, rl) != 0;
+                    if (tile_first_row + wq * 32 + rl >= p.Lq) continue;
+                    float* orow_k = obase + static_cast<size_t>(rl) * D + cp;
+                    const int h = k >> 1, up = k & 1;
+#pragma unroll
+                    for (int b = 0; b < D / 64; ++b) {
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int base = (h * (D / 64) + b) * 32 + 4 * c + 2 * up;
+                            const float x0 = zero ? 0.0f : __uint_as_float(ov[base]) * inv;
+                            const float x1 = zero ? 0.0f : __uint_as_float(ov[base + 1]) * inv;
+                            st_global_v2f(orow_k + b * 64 + 8 * c, x0, x1);
+                        }
+                    }
+                }
+                if (row < un.lq) p.lse[static_cast<size_t>(un.bh) * p.Lq + row] = m_ref * p.scale + logf(l);
+            } else {
                 // O leaves through the copy engine: per 128-byte column chunk, each
                 // thread writes its row's 128 bytes into the warp's 32-row stage in
                 // the 128-byte-swizzled layout of the O tensor map (16-byte pieces
