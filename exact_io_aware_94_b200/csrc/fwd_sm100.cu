@@ -81,10 +81,11 @@ struct FwdLayout {
     // drain[2]
     static constexpr int kNumBars = 4 + 4 * kStages + 10 + 2 + 2 * 4;  // + unit ring full/free
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    // unit ring: 4 unit indices, 4 int4 block-sparse metadata, 4 decoded units (32 bytes each)
+    static constexpr int kRingOff = kMiscOff + 16;
     // epilogue staging for the O tile stores: 4 KB per softmax warp (32 rows x 128 bytes,
     // 128-byte swizzle, so 1024-byte aligned)
-    static constexpr int kRingOff = kMiscOff + 16;  // 4 unit indices, then (block-sparse) 4 int4 unit metadata
-    static constexpr int kStageOff = (kRingOff + 16 + 64 + 1023) / 1024 * 1024;
+    static constexpr int kStageOff = (kRingOff + 16 + 64 + 128 + 1023) / 1024 * 1024;
     static constexpr int kBytes = kStageOff + 8 * 4096 + 1024;  // + alignment slack
 };
 
@@ -145,8 +146,8 @@ __device__ __forceinline__ Unit unit_of(const FwdParams& p, int u) {
 // sequence's end are empty (no KV tiles).  A sequence whose offsets are out of
 // range or decreasing, that is longer than max_pairs * 256 rows, that has
 // queries but no keys, or (causal) more queries than keys is skipped and
-// flagged FA_ERR_SEQLEN (once, by the producer, from its pair-0 unit).
-__device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u, bool flag) {
+// flagged FA_ERR_SEQLEN (once, from its pair-0 unit).
+__device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u) {
     const int BH = p.B * p.H;
     Unit r;
     const int pair = p.max_pairs - 1 - u / BH;
@@ -163,7 +164,7 @@ __device__ __forceinline__ Unit unit_of_varlen(const FwdParams& p, int u, bool f
     const bool bad = q0 < 0 || q1 < q0 || q1 > p.Lq || k0 < 0 || k1 < k0 || k1 > p.Lk ||
                      r.lq > p.max_pairs * kFwdRowsPerCta || (r.lq > 0 && r.lk == 0) || (p.causal && r.lq > r.lk);
     if (bad) {
-        if (flag && pair == 0) atomicCAS(p.status, 0, FA_ERR_SEQLEN);
+        if (pair == 0) atomicCAS(p.status, 0, FA_ERR_SEQLEN);
         r.lq = 0;
         return r;
     }
@@ -210,13 +211,37 @@ __device__ __forceinline__ const uint16_t* bsparse_list(const FwdParams& p, cons
     return p.bs_list + bsparse_index(p, un.bh, un.i0) * p.bs_tk;
 }
 
-// Unit u; block-sparse units need their metadata (meta), which the producer
-// reads once and publishes with the unit.
+// Unit u, decoded by the producer (block-sparse units need their metadata, meta);
+// the producer publishes it with the unit index.
 template <bool VARLEN, bool BSPARSE>
-__device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, bool flag, const int4& meta) {
-    if constexpr (VARLEN) return unit_of_varlen(p, u, flag);
+__device__ __forceinline__ Unit get_unit(const FwdParams& p, int u, const int4& meta) {
+    if constexpr (VARLEN) return unit_of_varlen(p, u);
     else if constexpr (BSPARSE) return unit_of_bsparse(p, u, meta);
     else return unit_of(p, u);
+}
+
+// A unit as published by the producer.  A batched unit's sequence fields are the
+// launch's own (0, 0, Lq, Lk): taking them from the parameters keeps them out of
+// the registers of the consumers' loops.
+template <bool VARLEN>
+__device__ __forceinline__ Unit read_unit(const FwdParams& p, const Unit* slot) {
+    Unit r;
+    r.bh = slot->bh;
+    r.i0 = slot->i0;
+    r.n_kv0 = slot->n_kv0;
+    r.n_kv1 = slot->n_kv1;
+    if constexpr (VARLEN) {
+        r.q0 = slot->q0;
+        r.k0 = slot->k0;
+        r.lq = slot->lq;
+        r.lk = slot->lk;
+    } else {
+        r.q0 = 0;
+        r.k0 = 0;
+        r.lq = p.Lq;
+        r.lk = p.Lk;
+    }
+    return r;
 }
 
 // The block-sparse metadata of unit u (read by the producer only).
@@ -273,6 +298,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
     uint64_t* bar_ufree = bar_ufull + kUnitRing;
     volatile int* s_unit = reinterpret_cast<volatile int*>(smem + Lay::kRingOff);
     int4* s_meta = reinterpret_cast<int4*>(smem + Lay::kRingOff + 16);  // block-sparse unit metadata
+    // The producer decodes each unit once and publishes it here.  The consumers' own
+    // decodes (integer divisions; for a packed batch, sequence offsets read from global
+    // memory) sat on the critical path at every unit boundary.
+    Unit* s_units = reinterpret_cast<Unit*>(smem + Lay::kRingOff + 80);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -361,12 +390,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                     u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
                     if (u >= n_units) break;
                     if constexpr (BSPARSE) meta = bsparse_meta_of(p, u);
-                    un = get_unit<VARLEN, BSPARSE>(p, u, true, meta);
+                    un = get_unit<VARLEN, BSPARSE>(p, u, meta);
                     if (!VARLEN || un.n_kv0 > 0 || un.n_kv1 > 0) break;
                 }
                 if (lane == 0) {
                     s_unit[rs] = u;
                     if constexpr (BSPARSE) s_meta[rs] = meta;
+                    if (u < n_units) s_units[rs] = un;
                     mbar_arrive(&bar_ufull[rs]);
                 }
                 __syncwarp();
@@ -478,10 +508,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 const int rs = it % kUnitRing;
                 if (!(ok = wait(&bar_ufull[rs], (it / kUnitRing) & 1))) break;
                 const int u = s_unit[rs];
+                const Unit un = read_unit<VARLEN>(p, &s_units[rs]);  // read before the slot is handed back
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
-                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, make_int4(0, 0, 0, 0));
                 const int n0 = un.n_kv0, n1 = un.n_kv1;
                 const int n_max = max(n0, n1);
                 if (!(ok = wait(&bar_k[kc % S], (kc / S) & 1))) break;
@@ -599,10 +629,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
                 if (!(ok = wait(&bar_ufull[rs], (it / kUnitRing) & 1))) break;
                 const int u = s_unit[rs];
                 const int4 meta = s_meta[rs];  // read before the slot is handed back
+                const Unit un = read_unit<VARLEN>(p, &s_units[rs]);
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ufree[rs]);
                 if (u >= n_units) break;
-                const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, meta);
                 // The unit's K/V tiles occupy ring positions kc .. kc + n_pos - 1; this
                 // warpgroup uses some of them (dense: the first n_w; block-sparse: the
                 // union-list entries with its bit), the last one at position `last`.
@@ -706,10 +736,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd_kernel(const __grid_con
             const int u = s_unit[rs];
             int4 meta = make_int4(0, 0, 0, 0);
             if constexpr (BSPARSE) meta = s_meta[rs];
+            const Unit un = read_unit<VARLEN>(p, &s_units[rs]);  // read before the slot is handed back
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit un = get_unit<VARLEN, BSPARSE>(p, u, false, meta);
             int n = (w == 0) ? un.n_kv0 : un.n_kv1;
             const uint16_t* bs_own = nullptr;  // block-sparse: this query block's own list
             if constexpr (BSPARSE) {
