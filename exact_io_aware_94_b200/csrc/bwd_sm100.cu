@@ -88,8 +88,8 @@ struct DkdvLayout {
     static constexpr int kGOff = kQOff + S * T::kTileBytes;         // dO, S stages
     static constexpr int kStatOff = kGOff + S * T::kTileBytes;      // per stage: lse2[128], dsum[128]
     static constexpr int kBarOff = kStatOff + S * 2 * 128 * 4;
-    // bars: kv, qd[S], empty[S], s, dp, p, ds, acc, drain
-    static constexpr int kNumBars = 1 + 2 * S + 6;
+    // bars: kv, qd[S], empty[S], s, dp, p, ds, acc, drain, p (second half)
+    static constexpr int kNumBars = 1 + 2 * S + 7;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16 + 1024;
 };
@@ -116,6 +116,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
     uint64_t* bar_ds = bar_s + 3;
     uint64_t* bar_acc = bar_s + 4;
     uint64_t* bar_drain = bar_s + 5;
+    // P^T is handed over in two halves of each warpgroup's 64 queries: bar_p for queries
+    // [0, 32), bar_p2 for [32, 64).  dV's MMAs on the first half run while the second
+    // half's exponentials are computed.
+    uint64_t* bar_p2 = bar_s + 6;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
         mbar_init(bar_p, 256);
+        mbar_init(bar_p2, 256);
         mbar_init(bar_ds, 256);
         mbar_init(bar_acc, 1);
         mbar_init(bar_drain, 1);
@@ -253,16 +258,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             for (int t = 0; ok && t < nq; ++t) {
                 const int s = t % S;
                 const bool more = t + 1 < nq;
-                // dV += P^T dO   (A = P^T from TMEM: queries 0-63 at cols [0,32), 64-127 at [64,96))
-                if (!(ok = wait(bar_p, t & 1))) break;
-                tc_fence_after();
+                // dV += P^T dO   (A = P^T from TMEM: queries 0-63 at cols [0,32), 64-127 at [64,96)),
+                // 16 queries per MMA: kk = 0, 1, 4, 5 take the first half of each warpgroup's
+                // queries (bar_p), kk = 2, 3, 6, 7 the second (bar_p2)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint32_t a = tmem_base + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
-                    umma_ts_w(tmem_base + kColDV, a,
-                              smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
-                              (t > 0 || kk > 0) ? 1u : 0u);
+                for (int h = 0; h < 2; ++h) {
+                    if (!(ok = wait(h == 0 ? bar_p : bar_p2, t & 1))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int kk = (i >> 1) * 4 + 2 * h + (i & 1);
+                        const uint32_t a = tmem_base + kColS + (kk >> 2) * 64 + (kk & 3) * 8;
+                        umma_ts_w(tmem_base + kColDV, a,
+                                  smem_desc_sw128(sGa + s * T::kTileBytes + kk * 2048, T::kBoxBytes, 1024), kIdescTS,
+                                  (t > 0 || kk > 0) ? 1u : 0u);
+                    }
                 }
+                if (!ok) break;
                 if (more) {
                     if (!(ok = wait(&bar_qd[(t + 1) % S], ((t + 1) / S) & 1))) break;
                     tc_fence_after();
@@ -325,21 +337,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv(const __grid_const
             }
             const float4* lse4 = reinterpret_cast<const float4*>(lse2);  // broadcast reads, 4 per load
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) {
-                const float4 lv = lse4[c4];
-                const float lc[4] = {lv.x, lv.y, lv.z, lv.w};
+            for (int h = 0; h < 2; ++h) {  // queries [32h, 32h + 32) of this warpgroup
 #pragma unroll
-                for (int x = 0; x < 4; ++x) pr[c4 * 4 + x] = ex2_approx(fmaf(pr[c4 * 4 + x], sl2, -lc[x]));
-            }
-            {
-                uint32_t pk[32];
+                for (int c4 = 8 * h; c4 < 8 * h + 8; ++c4) {
+                    const float4 lv = lse4[c4];
+                    const float lc[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-                tmem_st32(tS, pk);
+                    for (int x = 0; x < 4; ++x) pr[c4 * 4 + x] = ex2_approx(fmaf(pr[c4 * 4 + x], sl2, -lc[x]));
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[32 * h + 2 * c], pr[32 * h + 2 * c + 1]);
+                tmem_st16(tS + 16 * h, pk);
                 tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(h == 0 ? bar_p : bar_p2);
             }
-            tc_fence_before();
-            mbar_arrive(bar_p);
             ok = __all_sync(0xffffffffu, mbar_wait(bar_dp, t & 1, abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
