@@ -82,7 +82,9 @@ KERNEL_SOURCES = {
     "fa_fwd_kernel": ["fwd_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
     "fa_fwd256_kernel": ["fwd256_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
     "fa_bwd": ["bwd_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+    "fa_bwd256": ["bwd256_sm100.cu", "bwd_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
     "fa_decode": ["decode_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
+    "fa_decode_paged": ["decode_paged_mma.cu", "decode_sm100.cu", "ptx.cuh", "fa_internal.h", "api.cu"],
 }
 
 
@@ -531,6 +533,7 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
     legs["bwd_d256_L4096"] = {"ms": round(t_b256 * 1e3, 4), "TFLOP/s": round(fb256 / t_b256 / 1e12, 1),
                               "frac_of_peak": round(fb256 / t_b256 / 1e12 / peaks["bf16_tflops"], 4),
                               "launches": 3, "kernels": "fa_bwd_dot + fa_bwd_dkdv256 + fa_bwd_dq256",
+                              "traffic": recorded_traffic("fa_bwd256", "bwd_d256_L4096"),
                               "flops_convention": "2.5 x forward (5 GEMMs); the kernels run 9 (dK/dV halves "
                                                   "recompute S^T and dP^T; dQ recomputes S and dP)",
                               "config": "B4 H16 L4096 d256 causal"}
@@ -585,9 +588,13 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
         assert rc == fa.FA_OK
 
     fv = sum(attn_flops(1, Hv, int(n), int(n), dv_, True) for n in lens_v)
+    # algorithmic bytes: Q, K, V in (bf16), O (fp32) and LSE out
+    bytes_v = tot * Hv * dv_ * (3 * 2 + 4) + tot * Hv * 4
     t_v = time_steps(fwd_varlen, steps, warm, stream, dist, device) / steps
     legs["prefill_varlen"] = {"ms": round(t_v * 1e3, 4), "TFLOP/s": round(fv / t_v / 1e12, 1),
                               "frac_of_peak": round(fv / t_v / 1e12 / peaks["bf16_tflops"], 4), "launches": 1,
+                              "kernel": "fa_fwd_kernel (packed)",
+                              "traffic": recorded_traffic("fa_fwd_kernel", "prefill_varlen", bytes_v),
                               "config": "16 causal sequences, lengths U[512, 8192] (%d tokens), H16 d128, packed"
                                         % tot}
     del qv, kv_, vv, ov, lv
@@ -657,8 +664,8 @@ def run_legs(args, fa, torch, device, stream, peaks, peak_kind, rank, dist):
                                 "frac_of_peak": round(nbytes / t_p / 1e9 / peaks["hbm_gbs"], 4),
                                 "frac_of_nominal_8000": round(nbytes / t_p / 1e9 / NOMINAL_HBM_GBS, 4),
                                 "launches": 3,
-                                "kernels": "fa_decode_plan + fa_decode_paged_tma + fa_decode_combine",
-                                "traffic": recorded_traffic("fa_decode", "decode_paged_gqa", nbytes),
+                                "kernels": "fa_decode_plan + fa_decode_paged_mma + fa_decode_combine",
+                                "traffic": recorded_traffic("fa_decode_paged", "decode_paged_gqa", nbytes),
                                 "config": "B64 H32 Hkv8 (groups of 4) d128, 64-token pages in shuffled order, "
                                           "lengths U[1024, 32768]",
                                 "l2": "pages 2 x %.1f GiB, far larger than L2" % (kp.numel() * 2 / 2 ** 30)}
@@ -678,7 +685,9 @@ def run_profile_case(args, device):
     fwd256: the d = 256 forward at B=4 H=16 L=4,096;
     decode_paged_small: paged, grouped-head decode at B=16 H=32 Hkv=8;
     blocksparse_small: block-sparse causal forward at B=2 H=16 L=8192 with the
-    benchmark's mask recipe (192 MiB of Q/K/V, more than L2)."""
+    benchmark's mask recipe (192 MiB of Q/K/V, more than L2); blocksparse: the same at
+    the benchmark's B=2 H=16 L=16384; bwd256: forward then backward at B=4 H=16
+    L=4,096 d=256."""
     import torch
 
     import exact_io_aware_94_b200 as fa
@@ -721,11 +730,20 @@ def run_profile_case(args, device):
         for _ in range(calls):
             fa.forward_varlen(q, k, v, cu_d, cu_d, int(lens.max()), causal=True, stream=stream)
         nbytes = 0
-    elif args.profile_case == "blocksparse_small":
+    elif args.profile_case == "bwd256":
+        w = WORKLOADS["fwd_d256_L4096"]
+        B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+        q, k, v, g = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(4))
+        o, lse = fa.forward(q, k, v, causal=True, stream=stream)
+        ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), device)
+        for _ in range(calls):
+            fa.backward(q, k, v, o, g, lse, causal=True, ws=ws, stream=stream)
+        nbytes = 0
+    elif args.profile_case in ("blocksparse_small", "blocksparse"):
         from exact_io_aware_94_b200.inputs import blocksparse_mask
 
         w = WORKLOADS["prefill_blocksparse"]
-        B, H, L, d = 2, 16, 8192, 128
+        B, H, L, d = (2, 16, 8192, 128) if args.profile_case == "blocksparse_small" else (w["B"], w["H"], w["L"], w["d"])
         q, k, v = (torch.randn(B, H, L, d, generator=gen, device=device).to(torch.bfloat16) for _ in range(3))
         mask = blocksparse_mask(H, L, L, seed=w["seed"], sink=w["sink"], window=w["window"],
                                 p_random=w["p_random"]).to(device)
@@ -808,7 +826,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--ref-budget", type=float, default=5.0, help="seconds of oracle work per reference step")
     ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode_small", "varlen_small", "decode_paged_small",
-                                                    "blocksparse_small", "fwd256"],
+                                                    "blocksparse_small", "blocksparse", "fwd256", "bwd256"],
                     default=None,
                     help="run only this path W+K times for a profiler; no benchmark line")
     args = ap.parse_args(argv)
