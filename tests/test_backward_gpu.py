@@ -104,6 +104,40 @@ def test_backward_full_size_sampled_heads(cuda_device):
     assert rel_fro(dv_sum, g_sum) < 1e-2
 
 
+def test_backward_d256_full_size_sampled_heads(cuda_device):
+    """The d = 256 workload (B=4, H=16, L=4096, causal) as the benchmark times it;
+    the oracle runs the full backward of two heads, and properties that hold at
+    any size are checked on all."""
+    w = WORKLOADS["fwd_d256_L4096"]
+    B, H, L, d = w["B"], w["H"], w["L"], w["d"]
+    inp = attention_inputs(B, H, L, L, d, seed=w["seed"], q_scale=w["q_scale"], with_dO=True)
+    scale = 1.0 / math.sqrt(d)
+    dev = cuda_device
+    q, k, v, g = (t.to(dev) for t in (inp.q, inp.k, inp.v, inp.dO))
+    o, lse = fa.forward(q, k, v, scale=scale, causal=True)
+    ws = fa.workspace(fa.fa_backward_workspace_size(B, H, L, L, d), dev)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base = torch.cuda.memory_allocated()
+    dq, dk, dv = fa.backward(q, k, v, o, g, lse, scale=scale, causal=True, ws=ws)
+    torch.cuda.synchronize()
+    grown = torch.cuda.max_memory_allocated() - base
+    assert fa.fa_check_status() == fa.FA_OK
+    assert grown <= 3 * q.numel() * 2 + (1 << 20)  # the three gradients only
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all()
+    for (b, h) in ((0, 1), (B - 1, H - 2)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        dq_r, dk_r, dv_r, _ = oracle.backward(inp.q[sl], inp.k[sl], inp.v[sl], inp.dO[sl], scale, True)
+        check_grad(dq[sl], dq_r, "dQ b=%d h=%d" % (b, h))
+        check_grad(dk[sl], dk_r, "dK b=%d h=%d" % (b, h))
+        check_grad(dv[sl], dv_r, "dV b=%d h=%d" % (b, h))
+    # the sum over keys of dV equals the sum over queries of dO (the rows of P sum to 1)
+    dv_sum = dv.double().sum(dim=2).cpu().numpy()
+    g_sum = inp.dO.double().sum(dim=2).numpy()
+    assert rel_fro(dv_sum, g_sum) < 1e-2
+
+
 def test_backward_d256_determinism(cuda_device):
     """d = 256: two runs give bitwise identical gradients (no atomics)."""
     inp = attention_inputs(1, 2, 333, 333, 256, seed=19, with_dO=True)
