@@ -42,12 +42,13 @@ struct DkdvLay256 {
     static constexpr int kSmall = 64 * 64 * 2;         // box: 64 rows x 64 bf16 (8 KB)
     static constexpr int kKOff = 0;                    // K [128 keys][256], 4 boxes
     static constexpr int kVOff = kKOff + 4 * kBig;     // V
-    static constexpr int kQOff = kVOff + 4 * kBig;     // Q [64 queries][256], 4 boxes
-    static constexpr int kGOff = kQOff + 4 * kSmall;   // dO
-    static constexpr int kStatOff = kGOff + 4 * kSmall;  // lse2[64], dsum[64]
-    static constexpr int kBarOff = kStatOff + 2 * 64 * 4;
-    // kv, q, dO, qfree, dofree, s, dp, p, ds, acc, drain
-    static constexpr int kNumBars = 11;
+    static constexpr int kQStage = 4 * kSmall;         // Q [64 queries][256], 4 boxes
+    static constexpr int kQOff = kVOff + 4 * kBig;     // 2 stages
+    static constexpr int kGOff = kQOff + 2 * kQStage;  // dO, 1 stage
+    static constexpr int kStatOff = kGOff + 4 * kSmall;  // per Q stage: lse2[64], dsum[64]
+    static constexpr int kBarOff = kStatOff + 2 * 2 * 64 * 4;
+    // kv, q[2], dO, qfree[2], dofree, s, dp, p, ds, acc, drain
+    static constexpr int kNumBars = 13;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16 + 1024;
 };
@@ -62,17 +63,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
     uint8_t* sG = smem + Lay::kGOff;
     float* sStat = reinterpret_cast<float*>(smem + Lay::kStatOff);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
+    // Q tiles and their statistics are double-buffered: the next tile's copies and
+    // statistic loads run while this tile's MMAs and elementwise work do.  (Without that,
+    // each tile waited a full load after the previous tile's last MMA freed the buffer.)
     uint64_t* bar_kv = bars;         // K and V landed
-    uint64_t* bar_q = bars + 1;      // Q tile and its statistics landed
-    uint64_t* bar_do = bars + 2;     // dO tile landed
-    uint64_t* bar_qfree = bars + 3;  // S^T and dK MMAs are done with the Q tile (and its statistics)
-    uint64_t* bar_dofree = bars + 4; // dP^T and dV MMAs are done with the dO tile
-    uint64_t* bar_s = bars + 5;
-    uint64_t* bar_dp = bars + 6;
-    uint64_t* bar_p = bars + 7;
-    uint64_t* bar_ds = bars + 8;
-    uint64_t* bar_acc = bars + 9;
-    uint64_t* bar_drain = bars + 10;
+    uint64_t* bar_q = bars + 1;      // [stage]: Q tile and its statistics landed
+    uint64_t* bar_do = bars + 3;     // dO tile landed
+    uint64_t* bar_qfree = bars + 4;  // [stage]: S^T and dK MMAs are done with the Q tile (and its statistics)
+    uint64_t* bar_dofree = bars + 6; // dP^T and dV MMAs are done with the dO tile
+    uint64_t* bar_s = bars + 7;
+    uint64_t* bar_dp = bars + 8;
+    uint64_t* bar_p = bars + 9;
+    uint64_t* bar_ds = bars + 10;
+    uint64_t* bar_acc = bars + 11;
+    uint64_t* bar_drain = bars + 12;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -93,9 +97,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
 
     if (threadIdx.x == 0) {
         mbar_init(bar_kv, 1);
-        mbar_init(bar_q, 1 + 32);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(&bar_q[st], 1 + 32);
+            mbar_init(&bar_qfree[st], 1);
+        }
         mbar_init(bar_do, 1);
-        mbar_init(bar_qfree, 1);
         mbar_init(bar_dofree, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
@@ -131,19 +137,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
             kv_issued = true;
             for (int t = 0; t < nq; ++t) {
                 const int i0 = (qt0 + t) * 64;
-                if (t > 0 && !wait(bar_qfree, (t - 1) & 1)) break;
-                mbar_arrive_expect_tx_w(bar_q, 4 * Lay::kSmall);
-                for (int b = 0; b < 4; ++b) tma_load_3d_w(sQ + b * Lay::kSmall, &p.tm_q64, bar_q, b * 64, i0, bh);
+                const int qs = t & 1;
+                if (t >= 2 && !wait(&bar_qfree[qs], ((t >> 1) - 1) & 1)) break;
+                mbar_arrive_expect_tx_w(&bar_q[qs], Lay::kQStage);
+                for (int b = 0; b < 4; ++b)
+                    tma_load_3d_w(sQ + qs * Lay::kQStage + b * Lay::kSmall, &p.tm_q64, &bar_q[qs], b * 64, i0, bh);
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     const int r = lane * 2 + x;
                     const int i = i0 + r;
                     const bool valid = i < p.Lq;
                     const size_t idx = static_cast<size_t>(bh) * p.Lq + i;
-                    sStat[r] = valid ? p.lse[idx] * kLog2e : INFINITY;  // P = 0 for rows past Lq
-                    sStat[64 + r] = valid ? p.dsum[idx] : 0.0f;
+                    sStat[qs * 128 + r] = valid ? p.lse[idx] * kLog2e : INFINITY;  // P = 0 for rows past Lq
+                    sStat[qs * 128 + 64 + r] = valid ? p.dsum[idx] : 0.0f;
                 }
-                mbar_arrive(bar_q);
+                mbar_arrive(&bar_q[qs]);
                 ++issued_q;
                 if (t > 0 && !wait(bar_dofree, (t - 1) & 1)) break;
                 mbar_arrive_expect_tx_w(bar_do, 4 * Lay::kSmall);
@@ -153,7 +161,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
         }
         // every copy issued here lands before the CTA exits
         if (kv_issued) mbar_wait_drain(bar_kv, 0, p.status);
-        if (issued_q > 0) mbar_wait_drain(bar_q, (issued_q - 1) & 1, p.status);
+        for (int t = (issued_q > 2 ? issued_q - 2 : 0); t < issued_q; ++t)
+            mbar_wait_drain(&bar_q[t & 1], (t >> 1) & 1, p.status);
         if (issued_do > 0) mbar_wait_drain(bar_do, (issued_do - 1) & 1, p.status);
     } else if (warp == 9) {
         // ================= MMA issuer
@@ -187,9 +196,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
         bool ok = wait(bar_kv, 0);
         for (int t = 0; ok && t < nq; ++t) {
             // S^T(t) overwrites P^T(t-1) and dP^T(t) overwrites dS^T(t-1): both follow dK(t-1)
-            if (!(ok = wait(bar_q, t & 1))) break;
+            const uint32_t sQt = sQa + (t & 1) * Lay::kQStage;
+            if (!(ok = wait(&bar_q[t & 1], (t >> 1) & 1))) break;
             tc_fence_after();
-            issue_ss(kColS, sKa, sQa);
+            issue_ss(kColS, sKa, sQt);
             umma_commit_w(bar_s);
             if (!(ok = wait(bar_do, t & 1))) break;
             tc_fence_after();
@@ -201,8 +211,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
             umma_commit_w(bar_dofree);
             if (!(ok = wait(bar_ds, t & 1))) break;
             tc_fence_after();
-            issue_ts(kColDK, kColDP, sQa, t == 0);  // dK_h += dS^T Q[:, h]
-            umma_commit_w(bar_qfree);
+            issue_ts(kColDK, kColDP, sQt, t == 0);  // dK_h += dS^T Q[:, h]
+            umma_commit_w(&bar_qfree[t & 1]);
         }
         if (ok) umma_commit_w(bar_acc);
         umma_commit_w(bar_drain);
@@ -236,7 +246,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
                     if (key > i0 + c + off) pr[c] = -INFINITY;
             }
             // the statistics of tile t stay in place until its dK MMA is done
-            const float4* lse4 = reinterpret_cast<const float4*>(sStat + g * 32);
+            const float4* lse4 = reinterpret_cast<const float4*>(sStat + (t & 1) * 128 + g * 32);
 #pragma unroll
             for (int c4 = 0; c4 < 8; ++c4) {
                 const float4 lv = lse4[c4];
@@ -260,7 +270,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dkdv256(const __grid_co
                 uint32_t u[32], pk[16];
                 tmem_ld32(tDP, u);
                 tmem_wait_ld();
-                const float4* d4 = reinterpret_cast<const float4*>(sStat + 64 + g * 32);
+                const float4* d4 = reinterpret_cast<const float4*>(sStat + (t & 1) * 128 + 64 + g * 32);
 #pragma unroll
                 for (int c4 = 0; c4 < 8; ++c4) {
                     const float4 dv = d4[c4];
