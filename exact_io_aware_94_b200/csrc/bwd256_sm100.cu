@@ -333,11 +333,12 @@ struct DqLay256 {
     static constexpr int kSmall = 64 * 64 * 2;       // box: 64 rows x 64 bf16
     static constexpr int kQOff = 0;                  // Q [128 queries][256], 4 boxes
     static constexpr int kGOff = kQOff + 4 * kBig;   // dO
-    static constexpr int kKOff = kGOff + 4 * kBig;   // K [64 keys][256], 4 boxes
-    static constexpr int kVOff = kKOff + 4 * kSmall; // V
+    static constexpr int kKStage = 4 * kSmall;      // K [64 keys][256], 4 boxes
+    static constexpr int kKOff = kGOff + 4 * kBig;   // 2 stages
+    static constexpr int kVOff = kKOff + 2 * kKStage; // V, 1 stage
     static constexpr int kBarOff = kVOff + 4 * kSmall;
-    // qd, k, v, kfree, vfree, s, dp, dsr, acc, drain
-    static constexpr int kNumBars = 10;
+    // qd, k[2], v, kfree[2], vfree, s, dp, dsr, acc, drain
+    static constexpr int kNumBars = 12;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kBytes = kMiscOff + 16 + 1024;
 };
@@ -351,16 +352,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
     uint8_t* sK = smem + Lay::kKOff;
     uint8_t* sV = smem + Lay::kVOff;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBarOff);
+    // K tiles are double-buffered: a K tile is held until its dQ MMAs, the last of its
+    // key tile, so with one buffer the next tile's copy could only start after them.
     uint64_t* bar_qd = bars;         // Q and dO landed
-    uint64_t* bar_k = bars + 1;      // K tile landed
-    uint64_t* bar_v = bars + 2;      // V tile landed
-    uint64_t* bar_kfree = bars + 3;  // S and dQ MMAs are done with the K tile
-    uint64_t* bar_vfree = bars + 4;  // the dP MMAs are done with the V tile
-    uint64_t* bar_s = bars + 5;
-    uint64_t* bar_dp = bars + 6;
-    uint64_t* bar_dsr = bars + 7;
-    uint64_t* bar_acc = bars + 8;
-    uint64_t* bar_drain = bars + 9;
+    uint64_t* bar_k = bars + 1;      // [stage]: K tile landed
+    uint64_t* bar_v = bars + 3;      // V tile landed
+    uint64_t* bar_kfree = bars + 4;  // [stage]: S and dQ MMAs are done with the K tile
+    uint64_t* bar_vfree = bars + 6;  // the dP MMAs are done with the V tile
+    uint64_t* bar_s = bars + 7;
+    uint64_t* bar_dp = bars + 8;
+    uint64_t* bar_dsr = bars + 9;
+    uint64_t* bar_acc = bars + 10;
+    uint64_t* bar_drain = bars + 11;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
 
@@ -381,9 +384,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
 
     if (threadIdx.x == 0) {
         mbar_init(bar_qd, 1);
-        mbar_init(bar_k, 1);
+        for (int st = 0; st < 2; ++st) {
+            mbar_init(&bar_k[st], 1);
+            mbar_init(&bar_kfree[st], 1);
+        }
         mbar_init(bar_v, 1);
-        mbar_init(bar_kfree, 1);
         mbar_init(bar_vfree, 1);
         mbar_init(bar_s, 1);
         mbar_init(bar_dp, 1);
@@ -417,9 +422,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
             }
             qd_issued = true;
             for (int j = 0; j < nk; ++j) {
-                if (j > 0 && !wait(bar_kfree, (j - 1) & 1)) break;
-                mbar_arrive_expect_tx_w(bar_k, 4 * Lay::kSmall);
-                for (int b = 0; b < 4; ++b) tma_load_3d_w(sK + b * Lay::kSmall, &p.tm_k64, bar_k, b * 64, j * 64, bh);
+                const int ks = j & 1;
+                if (j >= 2 && !wait(&bar_kfree[ks], ((j >> 1) - 1) & 1)) break;
+                mbar_arrive_expect_tx_w(&bar_k[ks], Lay::kKStage);
+                for (int b = 0; b < 4; ++b)
+                    tma_load_3d_w(sK + ks * Lay::kKStage + b * Lay::kSmall, &p.tm_k64, &bar_k[ks], b * 64, j * 64, bh);
                 ++issued_k;
                 if (j > 0 && !wait(bar_vfree, (j - 1) & 1)) break;
                 mbar_arrive_expect_tx_w(bar_v, 4 * Lay::kSmall);
@@ -428,7 +435,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
             }
         }
         if (qd_issued) mbar_wait_drain(bar_qd, 0, p.status);
-        if (issued_k > 0) mbar_wait_drain(bar_k, (issued_k - 1) & 1, p.status);
+        for (int j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
+            mbar_wait_drain(&bar_k[j & 1], (j >> 1) & 1, p.status);
         if (issued_v > 0) mbar_wait_drain(bar_v, (issued_v - 1) & 1, p.status);
     } else if (warp == 9) {
         // ================= MMA issuer
@@ -450,9 +458,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
         bool ok = wait(bar_qd, 0);
         for (int j = 0; ok && j < nk; ++j) {
             // S(j) overwrites dS(j-1) and dP(j) overwrites dP(j-1): both follow dQ(j-1)
-            if (!(ok = wait(bar_k, j & 1))) break;
+            const uint32_t sKj = sKa + (j & 1) * Lay::kKStage;
+            if (!(ok = wait(&bar_k[j & 1], (j >> 1) & 1))) break;
             tc_fence_after();
-            issue_ss(kColS, sQa, sKa);
+            issue_ss(kColS, sQa, sKj);
             umma_commit_w(bar_s);
             if (!(ok = wait(bar_v, j & 1))) break;
             tc_fence_after();
@@ -466,10 +475,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) fa_bwd_dq256(const __grid_cons
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t a = tmem_base + kColS + (kk >> 1) * 32 + (kk & 1) * 8;
-                umma_ts_w(tmem_base + kColDQ, a, smem_desc_sw128(sKa + kk * 2048, Lay::kSmall, 1024), kIdescTS,
+                umma_ts_w(tmem_base + kColDQ, a, smem_desc_sw128(sKj + kk * 2048, Lay::kSmall, 1024), kIdescTS,
                           (j > 0 || kk > 0) ? 1u : 0u);
             }
-            umma_commit_w(bar_kfree);
+            umma_commit_w(&bar_kfree[j & 1]);
         }
         if (ok) umma_commit_w(bar_acc);
         umma_commit_w(bar_drain);
