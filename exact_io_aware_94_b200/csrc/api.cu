@@ -457,7 +457,7 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
                       const int* cu_seqlens_k, int B, int H, int total_q, int total_k, int max_seqlen_q, int d,
                       float scale, int causal, int o_dtype, void* stream) {
     if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (B <= 0 || H <= 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return FA_ERR_INVALID_ARG;
     if (!scale_ok(scale)) return FA_ERR_INVALID_ARG;
@@ -466,8 +466,10 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
         return FA_ERR_INVALID_ARG;
     if (static_cast<long long>(total_q) * H > 0x7FFFFFFFLL || static_cast<long long>(total_k) * H > 0x7FFFFFFFLL)
         return FA_ERR_INVALID_ARG;
-    const long long max_pairs = (static_cast<long long>(max_seqlen_q) + kFwdRowsPerCta - 1) / kFwdRowsPerCta;
-    if (static_cast<long long>(B) * H * max_pairs > 0x7FFFFFFFLL || max_pairs * kFwdRowsPerCta > 0x7FFFFFFFLL)
+    // units of 256 query rows (two 128-row tiles); at d = 256 single 128-row tiles
+    const int unit_rows = d == 256 ? kFwdBM : kFwdRowsPerCta;
+    const long long max_pairs = (static_cast<long long>(max_seqlen_q) + unit_rows - 1) / unit_rows;
+    if (static_cast<long long>(B) * H * max_pairs > 0x7FFFFFFFLL || max_pairs * unit_rows > 0x7FFFFFFFLL)
         return FA_ERR_INVALID_ARG;
     if (total_q == 0 || max_pairs == 0) return FA_OK;
     if (total_k == 0) return FA_ERR_INVALID_ARG;
@@ -477,8 +479,9 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
     if (rc != FA_OK) return rc;
     FwdParams p{};
     if ((rc = encode_packed_map_impl(&p.tm_q, q, total_q, H, d, kFwdBM, 2)) != FA_OK) return rc;
-    if ((rc = encode_packed_map_impl(&p.tm_k, k, total_k, H, d, kFwdBN, 2)) != FA_OK) return rc;
-    if ((rc = encode_packed_map_impl(&p.tm_v, v, total_k, H, d, kFwdBN, 2)) != FA_OK) return rc;
+    const int kv_rows = d == 256 ? kFwd256BN : kFwdBN;  // keys per K/V tile
+    if ((rc = encode_packed_map_impl(&p.tm_k, k, total_k, H, d, kv_rows, 2)) != FA_OK) return rc;
+    if ((rc = encode_packed_map_impl(&p.tm_v, v, total_k, H, d, kv_rows, 2)) != FA_OK) return rc;
     if ((rc = encode_packed_map_impl(&p.tm_o, o, total_q, H, d, 32, o_dtype == FA_DT_F32 ? 4 : 2)) != FA_OK)
         return rc;
     p.o = o;
@@ -496,7 +499,8 @@ int fa_forward_varlen(const void* q, const void* k, const void* v, void* o, floa
     p.scale_log2 = scale * 1.4426950408889634f;
     p.causal = causal ? 1 : 0;
     p.o_dtype = o_dtype;
-    cudaError_t e = launch_fwd_varlen(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
+    cudaError_t e = d == 256 ? launch_fwd256_varlen(p, st->num_sms, static_cast<cudaStream_t>(stream))
+                             : launch_fwd_varlen(p, d, st->num_sms, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

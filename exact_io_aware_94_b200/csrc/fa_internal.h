@@ -54,7 +54,8 @@ struct __align__(64) FwdParams {
                           // Null: static deal (no counters).
     // packed variable-length batch (fa_forward_varlen): sequence b owns rows [cu_q[b], cu_q[b+1])
     // of q, o [total_q, H, d] and [cu_k[b], cu_k[b+1]) of k, v [total_k, H, d]; Lq = total_q,
-    // Lk = total_k, and max_pairs = ceil(max_seqlen_q / 256).  Null for a batched call.
+    // Lk = total_k, and max_pairs = ceil(max_seqlen_q / 256) (d = 256: ceil(max_seqlen_q / 128),
+    // the kernel's units being single 128-row tiles).  Null for a batched call.
     const int* cu_q;
     const int* cu_k;
     int max_pairs;
@@ -204,6 +205,8 @@ cudaError_t launch_fwd(const FwdParams& p, int d, int num_sms, cudaStream_t stre
 // Head dimension 256: one 128-row Q tile per unit, K/V tiles of kFwd256BN keys.
 constexpr int kFwd256BN = 64;
 cudaError_t launch_fwd256(const FwdParams& p, int num_sms, cudaStream_t stream);
+// Packed batch at d = 256: p.max_pairs is the number of 128-row query tiles of the longest sequence.
+cudaError_t launch_fwd256_varlen(const FwdParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p, int d, int num_sms,
                                    cudaStream_t stream);

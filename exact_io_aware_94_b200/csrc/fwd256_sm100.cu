@@ -55,8 +55,9 @@ struct Lay256 {
     // q, q_free, k[S], v[S], kfree[S], vfree[S], s[2], p[2][2], pv, o, ofree, x[4], drain, ufull[R], ufree[R]
     static constexpr int kNumBars = 2 + 4 * kStages + 2 + 4 + 3 + 4 + 1 + 2 * kUnitRing;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    // unit ring: 4 unit indices, then 4 decoded units (32 bytes each)
     static constexpr int kRingOff = kMiscOff + 16;
-    static constexpr int kBytes = kRingOff + 16 + 1024;  // + alignment slack
+    static constexpr int kBytes = kRingOff + 16 + 128 + 1024;  // + alignment slack
 };
 
 // TMEM columns: S buffers [0, 64) and [64, 128); the partners' exchange slots
@@ -64,8 +65,13 @@ struct Lay256 {
 constexpr uint32_t kColX = 128;
 constexpr uint32_t kColO = 256;
 
-struct Unit256 {
-    int bh, i0, n;  // (b*H + h), first query row, 64-key tiles to visit
+// One work unit: (b*H + h), its first query row within the sequence, the 64-key tiles to
+// visit, and where its sequence lives (packed first rows and lengths; 0, 0, Lq, Lk for a
+// batched call).
+struct __align__(16) Unit256 {
+    int bh, i0, n;
+    int q0, k0, lq, lk;
+    int pad;
 };
 
 // Units in a fixed global order: the (b, h) pairs in groups of p.head_group heads
@@ -89,6 +95,45 @@ __device__ __forceinline__ Unit256 unit256_of(const FwdParams& p, int u) {
     } else {
         r.n = n_all;
     }
+    r.q0 = 0;
+    r.k0 = 0;
+    r.lq = p.Lq;
+    r.lk = p.Lk;
+    r.pad = 0;
+    return r;
+}
+
+// Packed variable-length batch: unit u is (query tile, b*H + h) in a virtual space of
+// p.max_pairs 128-row tiles per (b, h), longest causal rows first.  Units past a
+// sequence's end are empty (no KV tiles).  A sequence whose offsets are out of range or
+// decreasing, that is longer than max_pairs * 128 rows, that has queries but no keys, or
+// (causal) more queries than keys is skipped and flagged FA_ERR_SEQLEN (once, from its
+// tile-0 unit).
+__device__ __forceinline__ Unit256 unit256_of_varlen(const FwdParams& p, int u) {
+    const int BH = p.B * p.H;
+    Unit256 r;
+    const int qt = p.max_pairs - 1 - u / BH;
+    r.bh = u % BH;
+    r.i0 = qt * kBM;
+    r.n = 0;
+    r.pad = 0;
+    const int b = r.bh / p.H;
+    const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
+    r.q0 = q0;
+    r.k0 = k0;
+    r.lq = q1 - q0;
+    r.lk = k1 - k0;
+    const bool bad = q0 < 0 || q1 < q0 || q1 > p.Lq || k0 < 0 || k1 < k0 || k1 > p.Lk ||
+                     r.lq > p.max_pairs * kBM || (r.lq > 0 && r.lk == 0) || (p.causal && r.lq > r.lk);
+    if (bad) {
+        if (qt == 0) atomicCAS(p.status, 0, FA_ERR_SEQLEN);
+        r.lq = 0;
+        return r;
+    }
+    if (r.i0 < r.lq) {
+        const int n_all = (r.lk + kBN - 1) / kBN;
+        r.n = p.causal ? min(n_all, (min(r.i0 + kBM - 1, r.lq - 1) + r.lk - r.lq) / kBN + 1) : n_all;
+    }
     return r;
 }
 
@@ -102,6 +147,7 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     return __uint_as_float(r);
 }
 
+template <bool VARLEN>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_constant__ FwdParams p) {
     using Lay = Lay256;
     constexpr int S = kStages;
@@ -129,10 +175,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMiscOff + 4);
     volatile int* s_unit = reinterpret_cast<volatile int*>(smem + Lay::kRingOff);
+    // The producer decodes each unit once (for a packed batch that reads the sequence's
+    // offsets from global memory) and publishes it with the unit index.
+    Unit256* s_units = reinterpret_cast<Unit256*>(smem + Lay::kRingOff + 16);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int n_units = p.B * p.H * ((p.Lq + kBM - 1) / kBM);
+    const int n_units = p.B * p.H * (VARLEN ? p.max_pairs : (p.Lq + kBM - 1) / kBM);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -188,40 +237,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
         for (int it = 0; ok; ++it) {
             const int rs = it % kUnitRing;
             if (it >= kUnitRing && !(ok = wait(&bar_ufree[rs], ((it / kUnitRing) - 1) & 1))) break;
-            unsigned int ticket = 0;
-            if (p.sched) {
-                if (lane == 0) ticket = atomicAdd(p.sched, 1u);
-                ticket = __shfl_sync(0xffffffffu, ticket, 0);
-            } else {
-                const unsigned G = gridDim.x, k = claims++;
-                ticket = k * G + ((k & 1u) ? G - 1u - blockIdx.x : blockIdx.x);
+            int u;
+            Unit256 un;
+            for (;;) {  // a packed batch's virtual units past a sequence's end are skipped here
+                unsigned int ticket = 0;
+                if (p.sched) {
+                    if (lane == 0) ticket = atomicAdd(p.sched, 1u);
+                    ticket = __shfl_sync(0xffffffffu, ticket, 0);
+                } else {
+                    const unsigned G = gridDim.x, k = claims++;
+                    ticket = k * G + ((k & 1u) ? G - 1u - blockIdx.x : blockIdx.x);
+                }
+                u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
+                if (u >= n_units) break;
+                un = VARLEN ? unit256_of_varlen(p, u) : unit256_of(p, u);
+                if (!VARLEN || un.n > 0) break;
             }
-            const int u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
             if (lane == 0) {
                 s_unit[rs] = u;
+                if (u < n_units) s_units[rs] = un;
                 mbar_arrive(&bar_ufull[rs]);
             }
             __syncwarp();
             if (u >= n_units) break;
-            const Unit256 un = unit256_of(p, u);
             if (nq > 0 && !(ok = wait(bar_q_free, (nq - 1) & 1))) break;
             mbar_arrive_expect_tx_w(bar_q, Lay::kQBytes);
+            // batched maps are [B*H][L][d]; packed maps are [total][H][d]
             for (int b = 0; b < kD / 64; ++b)
-                tma_load_3d_w(sQ + b * Lay::kQBox, &p.tm_q, bar_q, b * 64, un.i0, un.bh);
+                tma_load_3d_w(sQ + b * Lay::kQBox, &p.tm_q, bar_q, b * 64, VARLEN ? un.bh % p.H : un.i0,
+                              VARLEN ? un.q0 + un.i0 : un.bh);
             ++nq;
             for (int j = 0; j < un.n; ++j, ++kc) {
                 const int s = kc % S;
                 if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
                 mbar_arrive_expect_tx_w(&bar_k[s], Lay::kKVBytes);
                 for (int b = 0; b < kD / 64; ++b)
-                    tma_load_3d_w(sK + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_k, &bar_k[s], b * 64, j * kBN,
-                                  un.bh);
+                    tma_load_3d_w(sK + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_k, &bar_k[s], b * 64,
+                                  VARLEN ? un.bh % p.H : j * kBN, VARLEN ? un.k0 + j * kBN : un.bh);
                 ++nk;
                 if (kc >= S && !(ok = wait(&bar_vfree[s], ((kc / S) - 1) & 1))) break;
                 mbar_arrive_expect_tx_w(&bar_v[s], Lay::kKVBytes);
                 for (int b = 0; b < kD / 64; ++b)
-                    tma_load_3d_w(sV + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_v, &bar_v[s], b * 64, j * kBN,
-                                  un.bh);
+                    tma_load_3d_w(sV + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_v, &bar_v[s], b * 64,
+                                  VARLEN ? un.bh % p.H : j * kBN, VARLEN ? un.k0 + j * kBN : un.bh);
                 ++nv;
             }
         }
@@ -265,11 +323,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             const int rs = it % kUnitRing;
             if (!(ok = wait(&bar_ufull[rs], (it / kUnitRing) & 1))) break;
             const int u = s_unit[rs];
+            const int n = s_units[rs].n;  // read before the slot is handed back
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit256 un = unit256_of(p, u);
-            const int n = un.n;
             if (!(ok = wait(bar_q, q_iter & 1))) break;
             ++q_iter;
             // the first two S of the unit (buffers of tiles ts and ts + 1)
@@ -324,7 +381,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
         const uint32_t lane_bits = static_cast<uint32_t>(wq * 32) << 16;
         const uint32_t t_row = tmem_base + lane_bits;
         const float sl2 = p.scale_log2;
-        const int off = p.Lk - p.Lq;  // causal: query i sits at key position i + off
         uint64_t* xbar = &bar_x[wq];
         int xc = 0;      // exchanges with the partner thread so far
         int ts = 0;      // tiles consumed
@@ -351,12 +407,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             ok = __all_sync(0xffffffffu, mbar_wait(&bar_ufull[rs], (it / kUnitRing) & 1, abort_flag, p.status));
             if (!ok) break;
             const int u = s_unit[rs];
+            Unit256 un;  // read before the slot is handed back
+            un.bh = s_units[rs].bh;
+            un.i0 = s_units[rs].i0;
+            un.n = s_units[rs].n;
+            if constexpr (VARLEN) {
+                un.q0 = s_units[rs].q0;
+                un.lq = s_units[rs].lq;
+                un.lk = s_units[rs].lk;
+            } else {
+                un.q0 = 0;
+                un.lq = p.Lq;
+                un.lk = p.Lk;
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_ufree[rs]);
             if (u >= n_units) break;
-            const Unit256 un = unit256_of(p, u);
-            const int row = un.i0 + row_in_tile;
-            const int limit = p.causal ? min(row + off, p.Lk - 1) : p.Lk - 1;  // highest permitted key
+            const int row = un.i0 + row_in_tile;  // within the sequence
+            const int off = un.lk - un.lq;        // causal: query i sits at key position i + off
+            const int limit = p.causal ? min(row + off, un.lk - 1) : un.lk - 1;  // highest permitted key
             float m_ref = -INFINITY;  // running max of raw scores (the same in both partners)
             float l = 0.0f;           // this thread's partial sum of the unrounded P~
             float corr = 0.0f;        // bf16 rounding of this half's largest P~, summed over tiles
@@ -468,11 +537,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
             const bool f32 = p.o_dtype == FA_DT_F32;
             const int n_chunks = f32 ? 4 : 2;  // 128-byte column chunks of this warpgroup's 128 columns
+            // A packed sequence's last partial 32-row box would spill into the next
+            // sequence's rows: its rows are written one by one instead.
+            const bool by_rows = VARLEN && un.i0 + wq * 32 + 32 > un.lq;
+            uint8_t* orow = nullptr;
+            if constexpr (VARLEN) {
+                const size_t esz = f32 ? 4 : 2;
+                orow = static_cast<uint8_t*>(p.o) + (static_cast<size_t>(un.q0 + row) * p.H + un.bh % p.H) * kD * esz +
+                       static_cast<size_t>(g) * 128 * esz;
+            }
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 if (k >= n_chunks) break;
-                if (lane == 0) bulk_wait_group_read0();  // the stage's previous store has read it
-                __syncwarp();
+                if (!by_rows) {
+                    if (lane == 0) bulk_wait_group_read0();  // the stage's previous store has read it
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     uint4 v;
@@ -489,17 +569,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
                         v.z = pack_bf16x2(__uint_as_float(ov[c0 + 4]) * inv, __uint_as_float(ov[c0 + 5]) * inv);
                         v.w = pack_bf16x2(__uint_as_float(ov[c0 + 6]) * inv, __uint_as_float(ov[c0 + 7]) * inv);
                     }
-                    *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
+                    if (by_rows) {
+                        if (row < un.lq) *reinterpret_cast<uint4*>(orow + k * 128 + q * 16) = v;
+                    } else {
+                        *reinterpret_cast<uint4*>(stg + lane * 128 + ((q ^ (lane & 7)) << 4)) = v;
+                    }
                 }
+                if (by_rows) continue;
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    if (un.i0 + wq * 32 < p.Lq)
-                        tma_store_3d(&p.tm_o, stg, g * 128 + k * (f32 ? 32 : 64), un.i0 + wq * 32, un.bh);
+                    if constexpr (VARLEN) {
+                        tma_store_3d(&p.tm_o, stg, g * 128 + k * (f32 ? 32 : 64), un.bh % p.H, un.q0 + un.i0 + wq * 32);
+                    } else {
+                        if (un.i0 + wq * 32 < p.Lq)
+                            tma_store_3d(&p.tm_o, stg, g * 128 + k * (f32 ? 32 : 64), un.i0 + wq * 32, un.bh);
+                    }
                     bulk_commit_group();
                 }
             }
-            if (g == 0 && row < p.Lq) p.lse[static_cast<size_t>(un.bh) * p.Lq + row] = m_ref * p.scale + logf(l_row);
+            // LSE: [B*H][Lq] for a batched call, [H][total_q] for a packed one
+            if (g == 0 && row < un.lq) {
+                const size_t li = VARLEN ? static_cast<size_t>(un.bh % p.H) * p.Lq + un.q0 + row
+                                         : static_cast<size_t>(un.bh) * p.Lq + row;
+                p.lse[li] = m_ref * p.scale + logf(l_row);
+            }
         }
     }
 
@@ -519,24 +613,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
     }
 }
 
+template <bool VARLEN>
+cudaError_t launch_fwd256_kernel(const FwdParams& p, int num_sms, cudaStream_t stream) {
+    const long long tiles = VARLEN ? p.max_pairs : (p.Lq + kBM - 1) / kBM;
+    const long long units = static_cast<long long>(p.B) * p.H * tiles;
+    if (units == 0) return cudaSuccess;
+    const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
+    cudaFuncAttributes a{};
+    cudaError_t e = cudaFuncGetAttributes(&a, fa_fwd256_kernel<VARLEN>);
+    if (e != cudaSuccess) return e;
+    // the setmaxnreg split must fit the registers the block is launched with
+    if (static_cast<long long>(a.numRegs) * kFwdThreads < 2LL * 128 * kFwdRegsSoftmax + 128LL * kFwdRegsOther)
+        return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(fa_fwd256_kernel<VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay256::kBytes);
+    if (e != cudaSuccess) return e;
+    fa_fwd256_kernel<VARLEN><<<grid, kFwdThreads, Lay256::kBytes, stream>>>(p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 int fwd256_smem_bytes() { return Lay256::kBytes; }
 
 cudaError_t launch_fwd256(const FwdParams& p, int num_sms, cudaStream_t stream) {
-    const long long units = static_cast<long long>(p.B) * p.H * ((p.Lq + kBM - 1) / kBM);
-    if (units == 0) return cudaSuccess;
-    const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
-    cudaFuncAttributes a{};
-    cudaError_t e = cudaFuncGetAttributes(&a, fa_fwd256_kernel);
-    if (e != cudaSuccess) return e;
-    // the setmaxnreg split must fit the registers the block is launched with
-    if (static_cast<long long>(a.numRegs) * kFwdThreads < 2LL * 128 * kFwdRegsSoftmax + 128LL * kFwdRegsOther)
-        return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(fa_fwd256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay256::kBytes);
-    if (e != cudaSuccess) return e;
-    fa_fwd256_kernel<<<grid, kFwdThreads, Lay256::kBytes, stream>>>(p);
-    return cudaGetLastError();
+    return launch_fwd256_kernel<false>(p, num_sms, stream);
+}
+
+// Packed batch: p.max_pairs is the number of 128-row query tiles of the longest sequence.
+cudaError_t launch_fwd256_varlen(const FwdParams& p, int num_sms, cudaStream_t stream) {
+    return launch_fwd256_kernel<true>(p, num_sms, stream);
 }
 
 }  // namespace fa

@@ -177,11 +177,13 @@ int fa_decode(const void* q, const void* kcache, const void* vcache, const int* 
  *   [cu_k[b], cu_k[b+1]), with cu[0] = 0 and cu[B] = total.
  *   max_seqlen_q >= every cu_q[b+1] - cu_q[b] (it sizes the work).
  *   o [total_q, H, d] (o_dtype), lse [H, total_q] fp32.
+ * d is 64, 128 or 256.
  * Causal masking is bottom-right per sequence (query i of a sequence sits at
  * key position i + Lk_b - Lq_b) and needs Lq_b <= Lk_b.  q, k, v, o must be
  * 16-byte aligned.  total_q = 0 returns FA_OK without a launch.  On the
  * device, a sequence whose offsets are out of range or decreasing, that is
- * longer than max_seqlen_q rounded up to 256, that has queries but no keys, or
+ * longer than max_seqlen_q rounded up to 256 (128 at d = 256), that has
+ * queries but no keys, or
  * (causal) more queries than keys is skipped (its rows are not written) and
  * flagged FA_ERR_SEQLEN in the status word.  Asynchronous on `stream`.
  */

@@ -35,7 +35,7 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("case", range(len(CASES)))
 def test_varlen_forward_parity(cuda_device, d, causal, case):
@@ -72,11 +72,12 @@ def test_varlen_many_sequences(cuda_device):
     check_lse(lse, lse_ref, "varlen LSE (40 sequences)")
 
 
-def test_varlen_invalid_sequence_is_skipped_and_flagged(cuda_device):
+@pytest.mark.parametrize("d", [64, 256])
+def test_varlen_invalid_sequence_is_skipped_and_flagged(cuda_device, d):
     """A causal sequence with more queries than keys is flagged and left unwritten;
     the other sequences are computed as usual."""
     lens_q, lens_k = [100, 50, 200], [100, 20, 200]  # sequence 1: 50 queries, 20 keys
-    H, d = 2, 64
+    H = 2
     inp = varlen_inputs(lens_q, lens_k, H, d, seed=8)
     o, lse = run(inp, H, d, True, torch.float32, cuda_device)
     assert fa.fa_check_status() == fa.FA_ERR_SEQLEN
