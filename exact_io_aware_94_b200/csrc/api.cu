@@ -330,7 +330,7 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
                            int H, int Lq, int Lk, int d, float scale, int causal, int o_dtype, void* workspace,
                            size_t workspace_bytes, void* stream) {
     if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
-    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
     if (o_dtype != FA_DT_BF16 && o_dtype != FA_DT_F32) return FA_ERR_UNSUPPORTED;
     if (!dims_ok(B, H, Lq, d) || !dims_ok(B, H, Lk, d)) return FA_ERR_INVALID_ARG;
     if (causal && Lq > Lk) return FA_ERR_INVALID_ARG;
@@ -370,8 +370,9 @@ int fa_forward_blocksparse(const void* q, const void* k, const void* v, void* o,
     FwdParams p{};
     const int BH = B * H;
     if ((rc = encode_rows_map(&p.tm_q, q, BH, Lq, d, kFwdBM)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
-    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kFwdBN)) != FA_OK) return rc;
+    const int kv_rows = d == 256 ? kFwd256BN : kFwdBN;  // keys per K/V tile
+    if ((rc = encode_rows_map(&p.tm_k, k, BH, Lk, d, kv_rows)) != FA_OK) return rc;
+    if ((rc = encode_rows_map(&p.tm_v, v, BH, Lk, d, kv_rows)) != FA_OK) return rc;
     if ((rc = encode_out_map_impl(&p.tm_o, o, BH, Lq, d, o_dtype)) != FA_OK) return rc;
     p.o = o;
     p.lse = lse;

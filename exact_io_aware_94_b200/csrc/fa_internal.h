@@ -207,6 +207,8 @@ constexpr int kFwd256BN = 64;
 cudaError_t launch_fwd256(const FwdParams& p, int num_sms, cudaStream_t stream);
 // Packed batch at d = 256: p.max_pairs is the number of 128-row query tiles of the longest sequence.
 cudaError_t launch_fwd256_varlen(const FwdParams& p, int num_sms, cudaStream_t stream);
+// Block-sparse batch at d = 256 (after the plan): p.bs_* set.
+cudaError_t launch_fwd256_blocksparse(const FwdParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_varlen(const FwdParams& p, int d, int num_sms, cudaStream_t stream);
 cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p, int d, int num_sms,
                                    cudaStream_t stream);

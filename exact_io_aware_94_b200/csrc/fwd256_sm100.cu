@@ -66,12 +66,12 @@ constexpr uint32_t kColX = 128;
 constexpr uint32_t kColO = 256;
 
 // One work unit: (b*H + h), its first query row within the sequence, the 64-key tiles to
-// visit, and where its sequence lives (packed first rows and lengths; 0, 0, Lq, Lk for a
-// batched call).
+// visit, where its sequence lives (packed first rows and lengths; 0, 0, Lq, Lk for a
+// batched call), and (block-sparse) the index of its query block's own key-block list.
 struct __align__(16) Unit256 {
     int bh, i0, n;
     int q0, k0, lq, lk;
-    int pad;
+    int lst;
 };
 
 // Units in a fixed global order: the (b, h) pairs in groups of p.head_group heads
@@ -99,7 +99,22 @@ __device__ __forceinline__ Unit256 unit256_of(const FwdParams& p, int u) {
     r.k0 = 0;
     r.lq = p.Lq;
     r.lk = p.Lk;
-    r.pad = 0;
+    r.lst = 0;
+    return r;
+}
+
+// Block-sparse: the batched unit order; the unit's 128-row query block visits the key
+// blocks of its own list (planned before the launch for pairs of query blocks, at least
+// one entry), each as two 64-key tiles.
+__device__ __forceinline__ Unit256 unit256_of_bsparse(const FwdParams& p, int u) {
+    Unit256 r = unit256_of(p, u);
+    const int qb = r.i0 / kBM;
+    const int n_pairs = (p.Lq + 2 * kBM - 1) / (2 * kBM);
+    const int ui = r.bh * n_pairs + (qb >> 1);
+    const int w = qb & 1;
+    const int cnt = (__ldg(p.bs_meta + ui).w >> (16 * w)) & 0xffff;
+    r.n = 2 * cnt;
+    r.lst = 2 * ui + w;
     return r;
 }
 
@@ -116,7 +131,7 @@ __device__ __forceinline__ Unit256 unit256_of_varlen(const FwdParams& p, int u) 
     r.bh = u % BH;
     r.i0 = qt * kBM;
     r.n = 0;
-    r.pad = 0;
+    r.lst = 0;
     const int b = r.bh / p.H;
     const int q0 = p.cu_q[b], q1 = p.cu_q[b + 1], k0 = p.cu_k[b], k1 = p.cu_k[b + 1];
     r.q0 = q0;
@@ -147,7 +162,7 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     return __uint_as_float(r);
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool BSPARSE>
 __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_constant__ FwdParams p) {
     using Lay = Lay256;
     constexpr int S = kStages;
@@ -250,7 +265,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
                 }
                 u = static_cast<int>(min(ticket, static_cast<unsigned>(n_units)));
                 if (u >= n_units) break;
-                un = VARLEN ? unit256_of_varlen(p, u) : unit256_of(p, u);
+                if constexpr (VARLEN) un = unit256_of_varlen(p, u);
+                else if constexpr (BSPARSE) un = unit256_of_bsparse(p, u);
+                else un = unit256_of(p, u);
                 if (!VARLEN || un.n > 0) break;
             }
             if (lane == 0) {
@@ -267,19 +284,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
                 tma_load_3d_w(sQ + b * Lay::kQBox, &p.tm_q, bar_q, b * 64, VARLEN ? un.bh % p.H : un.i0,
                               VARLEN ? un.q0 + un.i0 : un.bh);
             ++nq;
+            const uint16_t* own = BSPARSE ? p.bs_own + static_cast<size_t>(un.lst) * p.bs_tk : nullptr;
             for (int j = 0; j < un.n; ++j, ++kc) {
                 const int s = kc % S;
+                int ky = j * kBN;  // first key of the tile (batched and block-sparse maps)
+                if constexpr (BSPARSE) ky = (__ldg(own + (j >> 1)) & kBsEntryTile) * (2 * kBN) + (j & 1) * kBN;
                 if (kc >= S && !(ok = wait(&bar_kfree[s], ((kc / S) - 1) & 1))) break;
                 mbar_arrive_expect_tx_w(&bar_k[s], Lay::kKVBytes);
                 for (int b = 0; b < kD / 64; ++b)
                     tma_load_3d_w(sK + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_k, &bar_k[s], b * 64,
-                                  VARLEN ? un.bh % p.H : j * kBN, VARLEN ? un.k0 + j * kBN : un.bh);
+                                  VARLEN ? un.bh % p.H : ky, VARLEN ? un.k0 + j * kBN : un.bh);
                 ++nk;
                 if (kc >= S && !(ok = wait(&bar_vfree[s], ((kc / S) - 1) & 1))) break;
                 mbar_arrive_expect_tx_w(&bar_v[s], Lay::kKVBytes);
                 for (int b = 0; b < kD / 64; ++b)
                     tma_load_3d_w(sV + s * Lay::kKVBytes + b * Lay::kKVBox, &p.tm_v, &bar_v[s], b * 64,
-                                  VARLEN ? un.bh % p.H : j * kBN, VARLEN ? un.k0 + j * kBN : un.bh);
+                                  VARLEN ? un.bh % p.H : ky, VARLEN ? un.k0 + j * kBN : un.bh);
                 ++nv;
             }
         }
@@ -411,6 +431,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             un.bh = s_units[rs].bh;
             un.i0 = s_units[rs].i0;
             un.n = s_units[rs].n;
+            un.lst = BSPARSE ? s_units[rs].lst : 0;
             if constexpr (VARLEN) {
                 un.q0 = s_units[rs].q0;
                 un.lq = s_units[rs].lq;
@@ -429,8 +450,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             float m_ref = -INFINITY;  // running max of raw scores (the same in both partners)
             float l = 0.0f;           // this thread's partial sum of the unrounded P~
             float corr = 0.0f;        // bf16 rounding of this half's largest P~, summed over tiles
+            const uint16_t* own = BSPARSE ? p.bs_own + static_cast<size_t>(un.lst) * p.bs_tk : nullptr;
             for (int j = 0; j < un.n; ++j, ++ts) {
                 const int b = ts & 1;
+                int bs_entry = 0;  // issued before the wait, used after it
+                if constexpr (BSPARSE) bs_entry = __ldg(own + (j >> 1));
                 ok = __all_sync(0xffffffffu, mbar_wait(&bar_s[b], (ts >> 1) & 1, abort_flag, p.status));
                 if (!ok) break;
                 tc_fence_after();
@@ -442,11 +466,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
 #pragma unroll
                     for (int x = 0; x < 32; ++x) s[x] = __uint_as_float(r[x]);
                 }
-                const int kv0 = j * kBN + g * 32;
-                if (kv0 + 31 > limit) {
+                int kv0 = j * kBN + g * 32;
+                bool mine = true;  // block-sparse: this query block may see the tile
+                if constexpr (BSPARSE) {
+                    kv0 = (bs_entry & kBsEntryTile) * (2 * kBN) + (j & 1) * kBN + g * 32;
+                    mine = !(bs_entry & kBsOwnMasked);
+                }
+                const int lim = mine ? limit : kv0 - 1;  // a tile it may not see is masked whole
+                if (kv0 + 31 > lim) {
 #pragma unroll
                     for (int c = 0; c < 32; ++c)
-                        if (kv0 + c > limit) s[c] = -INFINITY;
+                        if (kv0 + c > lim) s[c] = -INFINITY;
                 }
                 float mx;
                 {
@@ -518,7 +548,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             if (!(ok = __all_sync(0xffffffffu, exchange(l, l_other)))) break;
             if (!(ok = __all_sync(0xffffffffu, exchange(corr, c_other)))) break;
             const float l_row = l + l_other;
-            const float inv = 1.0f / (l_row + corr + c_other);
+            const float den = l_row + corr + c_other;
+            // Block-sparse: a row that may see no key has l = 0 and gets O = 0, LSE = -inf.
+            const bool empty_row = BSPARSE && !(den > 0.0f);
+            const float inv = empty_row ? 0.0f : 1.0f / den;
             ok = __all_sync(0xffffffffu, mbar_wait(bar_o, units & 1, abort_flag, p.status));
             if (!ok) break;
             ++units;
@@ -534,6 +567,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(bar_ofree);  // O may now be overwritten by the next unit's PV
+            if constexpr (BSPARSE) {
+                // Cleared rather than scaled: the fully masked tile such a row ran may hold
+                // non-finite V rows, and 0 * inf or 0 * NaN in the PV product is NaN.
+                if (empty_row) {
+#pragma unroll
+                    for (int c = 0; c < 128; ++c) ov[c] = 0u;
+                }
+            }
             uint8_t* stg = smem + Lay::kStageOff + warp * 4096;
             const bool f32 = p.o_dtype == FA_DT_F32;
             const int n_chunks = f32 ? 4 : 2;  // 128-byte column chunks of this warpgroup's 128 columns
@@ -613,21 +654,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1) fa_fwd256_kernel(const __grid_
     }
 }
 
-template <bool VARLEN>
+template <bool VARLEN, bool BSPARSE>
 cudaError_t launch_fwd256_kernel(const FwdParams& p, int num_sms, cudaStream_t stream) {
     const long long tiles = VARLEN ? p.max_pairs : (p.Lq + kBM - 1) / kBM;
     const long long units = static_cast<long long>(p.B) * p.H * tiles;
     if (units == 0) return cudaSuccess;
     const dim3 grid(static_cast<unsigned>(units < num_sms ? units : num_sms));
     cudaFuncAttributes a{};
-    cudaError_t e = cudaFuncGetAttributes(&a, fa_fwd256_kernel<VARLEN>);
+    cudaError_t e = cudaFuncGetAttributes(&a, fa_fwd256_kernel<VARLEN, BSPARSE>);
     if (e != cudaSuccess) return e;
     // the setmaxnreg split must fit the registers the block is launched with
     if (static_cast<long long>(a.numRegs) * kFwdThreads < 2LL * 128 * kFwdRegsSoftmax + 128LL * kFwdRegsOther)
         return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(fa_fwd256_kernel<VARLEN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay256::kBytes);
+    e = cudaFuncSetAttribute(fa_fwd256_kernel<VARLEN, BSPARSE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Lay256::kBytes);
     if (e != cudaSuccess) return e;
-    fa_fwd256_kernel<VARLEN><<<grid, kFwdThreads, Lay256::kBytes, stream>>>(p);
+    fa_fwd256_kernel<VARLEN, BSPARSE><<<grid, kFwdThreads, Lay256::kBytes, stream>>>(p);
     return cudaGetLastError();
 }
 
@@ -636,12 +678,17 @@ cudaError_t launch_fwd256_kernel(const FwdParams& p, int num_sms, cudaStream_t s
 int fwd256_smem_bytes() { return Lay256::kBytes; }
 
 cudaError_t launch_fwd256(const FwdParams& p, int num_sms, cudaStream_t stream) {
-    return launch_fwd256_kernel<false>(p, num_sms, stream);
+    return launch_fwd256_kernel<false, false>(p, num_sms, stream);
 }
 
 // Packed batch: p.max_pairs is the number of 128-row query tiles of the longest sequence.
 cudaError_t launch_fwd256_varlen(const FwdParams& p, int num_sms, cudaStream_t stream) {
-    return launch_fwd256_kernel<true>(p, num_sms, stream);
+    return launch_fwd256_kernel<true, false>(p, num_sms, stream);
+}
+
+// Block-sparse batch (the plan has run on the stream before): p.bs_* set.
+cudaError_t launch_fwd256_blocksparse(const FwdParams& p, int num_sms, cudaStream_t stream) {
+    return launch_fwd256_kernel<false, true>(p, num_sms, stream);
 }
 
 }  // namespace fa

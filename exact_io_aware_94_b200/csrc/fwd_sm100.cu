@@ -1155,6 +1155,7 @@ cudaError_t launch_fwd_blocksparse(const BsPlanParams& plan, const FwdParams& p,
     fa_bsparse_plan<<<static_cast<unsigned>(blocks), kBsPlanThreads, 0, stream>>>(plan);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (d == 256) return launch_fwd256_blocksparse(p, num_sms, stream);
     return d == 128 ? launch_fwd_kernel<128, false, true>(p, num_sms, stream)
                     : launch_fwd_kernel<64, false, true>(p, num_sms, stream);
 }

@@ -240,7 +240,7 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
  * would permit it (length bound, causal mask) AND its block byte is nonzero;
  * the result is the exact softmax attention over the permitted keys.  A row
  * with no permitted key gets O = 0 and LSE = -inf.
- *   q, k, v, o, lse, scale, causal, o_dtype: as fa_forward.
+ *   q, k, v, o, lse, scale, causal, o_dtype: as fa_forward (d is 64, 128 or 256).
  *   block_mask: DEVICE bytes; the mask of (b, h) is row-major [Tq][Tk] at
  *   block_mask + b * mask_stride_b + h * mask_stride_h, with
  *   Tq = ceil(Lq / 128), Tk = ceil(Lk / 128); strides are in bytes, >= 0
@@ -251,7 +251,8 @@ int fa_decode_paged(const void* q, const void* kpages, const void* vpages, const
  *   the per-unit lists of key blocks that a small planning kernel builds
  *   before the forward kernel (both launched on `stream`).
  * Blocks whose byte is zero cost no tensor-core work unless the other
- * 128-row query block that shares a 256-row work unit needs them.
+ * 128-row query block that shares a 256-row work unit needs them (at d = 256
+ * a work unit is a single query block).
  */
 #define FA_BLOCKSPARSE_BLOCK 128
 size_t fa_forward_blocksparse_workspace_size(int B, int H, int Lq, int Lk);

@@ -37,11 +37,12 @@ def run_both(inp, mask_dev, mask_np, causal, dev, what):
     return o_ref, lse_ref
 
 
+@pytest.mark.parametrize("d", [128, 256])
 @pytest.mark.parametrize("causal", [True, False])
-def test_all_ones_mask_equals_dense_forward_bitwise(cuda_device, causal):
+def test_all_ones_mask_equals_dense_forward_bitwise(cuda_device, causal, d):
     """With every block permitted each query block walks the same key tiles as in the dense
     forward, in the same order, with the same arithmetic: bit-identical output."""
-    B, H, L, d = 1, 2, 700, 128
+    B, H, L = 1, 2, 700
     inp = attention_inputs(B, H, L, L, d, seed=50)
     q, k, v = inp.q.to(cuda_device), inp.k.to(cuda_device), inp.v.to(cuda_device)
     ones = torch.ones(tiles(L), tiles(L), dtype=torch.uint8, device=cuda_device)
@@ -51,7 +52,7 @@ def test_all_ones_mask_equals_dense_forward_bitwise(cuda_device, causal):
     assert torch.equal(o, od) and torch.equal(lse, ld)
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("Lq,Lk", [(300, 520), (513, 129), (1000, 1000)])
 def test_random_per_head_masks_noncausal(cuda_device, d, Lq, Lk):
     """A different random mask per (b, h) (density 1/2), ragged lengths on both sides."""
@@ -62,7 +63,7 @@ def test_random_per_head_masks_noncausal(cuda_device, d, Lq, Lk):
     run_both(inp, torch.from_numpy(mask).to(cuda_device), mask, False, cuda_device, "random masks")
 
 
-@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("Lq,Lk", [(1000, 1000), (384, 900)])
 def test_sink_window_random_causal(cuda_device, d, Lq, Lk):
     """The benchmark's pattern (sink, local window, random blocks below the diagonal), one mask
@@ -73,10 +74,11 @@ def test_sink_window_random_causal(cuda_device, d, Lq, Lk):
     run_both(inp, mask.to(cuda_device), mask.numpy(), True, cuda_device, "sink/window/random")
 
 
-def test_rows_with_no_key_are_zero_with_lse_minus_inf(cuda_device):
+@pytest.mark.parametrize("d", [128, 256])
+def test_rows_with_no_key_are_zero_with_lse_minus_inf(cuda_device, d):
     """Query blocks whose mask row is empty -- one block of a pair, and a whole 256-row unit --
     get O = 0 and LSE = -inf; so does a causal row block permitted only above its diagonal."""
-    B, H, L, d = 1, 2, 900, 128
+    B, H, L = 1, 2, 900
     inp = attention_inputs(B, H, L, L, d, seed=53)
     t = tiles(L)
     mask = np.ones((H, t, t), np.uint8)
@@ -91,11 +93,12 @@ def test_rows_with_no_key_are_zero_with_lse_minus_inf(cuda_device):
     assert (o[0, 1, 256:512] == 0).all() and torch.isneginf(lse[0, 1, 640:768]).all()
 
 
-def test_blocks_nobody_sees_hold_nan(cuda_device):
+@pytest.mark.parametrize("d", [128, 256])
+def test_blocks_nobody_sees_hold_nan(cuda_device, d):
     """K/V rows of key blocks that no query block may see are NaN.  A unit whose two query
     blocks see nothing still runs one fully masked tile, which may be such a block: its rows
     must still be exactly 0 with LSE = -inf, and every other row must match the oracle."""
-    B, H, L, d = 1, 2, 640, 128
+    B, H, L = 1, 2, 640
     inp = attention_inputs(B, H, L, L, d, seed=56)
     t = tiles(L)
     mask = np.zeros((H, t, t), np.uint8)
@@ -114,11 +117,12 @@ def test_blocks_nobody_sees_hold_nan(cuda_device):
     check_lse(lse, lse_ref, "NaN in unseen blocks")
 
 
+@pytest.mark.parametrize("d", [64, 256])
 @pytest.mark.parametrize("causal", [True, False])
-def test_all_zero_mask(cuda_device, causal):
+def test_all_zero_mask(cuda_device, causal, d):
     """No block permitted anywhere: every unit runs only its one fully masked entry, and every
     row gets O = 0 and LSE = -inf, in both output types."""
-    B, H, L, d = 2, 2, 333, 64
+    B, H, L = 2, 2, 333
     inp = attention_inputs(B, H, L, L, d, seed=57)
     zeros = torch.zeros(tiles(L), tiles(L), dtype=torch.uint8, device=cuda_device)
     for out_dtype in (torch.float32, torch.bfloat16):
