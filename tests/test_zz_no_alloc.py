@@ -30,6 +30,7 @@ def _noalloc(q, k, v, o, g, lse, B, H, Lq, Lk, d, scale, causal, o_dtype):
     (64, 700, 700, True, torch.bfloat16),
     (128, 300, 650, True, torch.bfloat16),   # fewer queries than keys: bottom-right causal
     (64, 257, 513, False, torch.float32),
+    (256, 300, 300, True, torch.float32),
 ])
 def test_noalloc_backward_matches_workspace_backward_twice(cuda_device, d, Lq, Lk, causal, out_dtype):
     dev = cuda_device
