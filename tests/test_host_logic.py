@@ -49,3 +49,26 @@ def test_blocksparse_mask_recipe():
     # bottom-right reach when Lq < Lk: query block r reaches key block r + (Lk - Lq) / 128
     m2 = blocksparse_mask(1, 256, 1024, seed=1, sink=0, window=1, p_random=0.0)
     assert m2[0].tolist() == [[0, 0, 0, 0, 0, 0, 1, 0], [0, 0, 0, 0, 0, 0, 0, 1]]
+
+
+def test_traffic_records_match_their_capture_summaries():
+    """Every DRAM-traffic record the benchmark can report names a committed ncu summary that
+    states the same kernel-source hash, and its kernel family is one the benchmark hashes."""
+    import json
+    import os
+    import re
+
+    import bench
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    with open(os.path.join(root, "profiles", "traffic.json")) as fh:
+        rec = json.load(fh)
+    assert rec
+    for kernel, workloads in rec.items():
+        assert kernel in bench.KERNEL_SOURCES, kernel
+        for workload, e in workloads.items():
+            assert ("bytes_per_launch" in e) != ("traffic_over_algorithmic" in e), (kernel, workload)
+            with open(os.path.join(root, e["capture"])) as fh:
+                text = fh.read()
+            m = re.search(r"Kernel source state: hash `([0-9a-f]{16})`", text)
+            assert m and m.group(1) == e["source_hash"], (kernel, workload, e["capture"])
